@@ -1,0 +1,406 @@
+"""Pins of the fp64 oracle against things other than itself: closed forms,
+invariants, an independent library routine (torch's scaled-dot-product
+attention in fp64 with an explicit block-causal mask), brute force over drop
+sets, and planted mistakes that must trip at least one pin."""
+from fractions import Fraction
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import attention as oatt
+from synth import SIDES_TINY, bf16_bits_to_f32, normal_bf16_bits, derive_key, gen_tau, gen_bias
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _qkv(B, H, T, D, tag=0):
+    out = []
+    for which in range(3):
+        bits = normal_bf16_bits(derive_key(99, tag, which), (B, H, T, D))
+        out.append(bf16_bits_to_f32(bits).astype(np.float64))
+    return out
+
+
+def _geom(sides):
+    return oracle.ScaleGeometry(sides)
+
+
+# ---------------------------------------------------------------- attention
+
+def test_mass_rows_sum_to_one_and_scas_column_sums():
+    """Every softmax row sums to 1, so sum_{s<=k} M[h][s][k] = 1 per scale."""
+    sides = SIDES_TINY
+    g = _geom(sides)
+    q, k, v = _qkv(2, 3, g.T, 64)
+    tau = gen_tau(1, 3).astype(np.float64)
+    bias = gen_bias(1, 3, g.S).astype(np.float64)
+    _, mass = oracle.block_causal_attention(q, k, v, sides, tau, bias)
+    np.testing.assert_allclose(mass.sum(axis=3), 1.0, atol=1e-12, rtol=0)
+    M = oracle.scas_mass(mass, sides)
+    for kk in range(g.S):
+        np.testing.assert_allclose(M[:, :kk + 1, kk].sum(axis=1), 1.0, atol=1e-12, rtol=0)
+        assert np.all(M[:, kk + 1:, kk] == 0.0)
+
+
+def _read_uniform_golden():
+    vals = {}
+    with open(os.path.join(GOLDEN, "uniform_scas_tiny.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            s, expr = line.split()
+            total = Fraction(0)
+            for term in expr.split("+"):
+                total += Fraction(term)
+            vals[int(s)] = total
+    return vals
+
+
+def test_uniform_attention_closed_form_golden():
+    """Q = 0, no bias: M[s][k] = n_s / L_k and S-CAS from the golden fixture."""
+    sides = SIDES_TINY
+    g = _geom(sides)
+    _, k, v = _qkv(2, 2, g.T, 64, tag=1)
+    q = np.zeros_like(k)
+    tau = np.array([0.7, 1.9])
+    _, mass = oracle.block_causal_attention(q, k, v, sides, tau, None)
+    M = oracle.scas_mass(mass, sides)
+    for kk in range(g.S):
+        for s in range(kk + 1):
+            assert abs(M[0, s, kk] - g.n[s] / g.L[kk]) < 1e-14
+    scas = oracle.scas_from_mass(M[None])[0]
+    gold = _read_uniform_golden()
+    for s, val in gold.items():
+        np.testing.assert_allclose(scas[:, s], float(val), atol=1e-14, rtol=0)
+    # the golden file's first row written out as the project-page example
+    assert abs(float(gold[0]) - (1/5 + 1/14 + 1/30 + 1/55 + 1/91 + 1/155)) < 1e-15
+
+
+def test_bias_only_closed_form():
+    """Q = 0 with a per-scale logit bias: M[s][k] = n_s e^b_s / sum_{s'<=k} n_s' e^b_s'."""
+    sides = SIDES_TINY
+    g = _geom(sides)
+    _, k, v = _qkv(1, 2, g.T, 64, tag=2)
+    q = np.zeros_like(k)
+    bias = np.array([[0.3, 1.7, 0.0, 2.0, 0.5, 0.0, 1.1], [0, 0, 1.5, 0, 0, 0, 0.2]])
+    _, mass = oracle.block_causal_attention(q, k, v, sides, np.array([1.0, 1.3]), bias)
+    M = oracle.scas_mass(mass, sides)
+    for h in range(2):
+        for kk in range(g.S):
+            den = sum(g.n[s] * math.exp(bias[h][s]) for s in range(kk + 1))
+            for s in range(kk + 1):
+                assert abs(M[h, s, kk] - g.n[s] * math.exp(bias[h][s]) / den) < 1e-13
+
+
+def test_scale_indicator_values_reproduce_mass():
+    """V columns set to scale indicators: O[:, s] equals the row mass m_i(s)."""
+    sides = SIDES_TINY
+    g = _geom(sides)
+    q, k, _ = _qkv(1, 2, g.T, 64, tag=3)
+    v = np.zeros((1, 2, g.T, g.S))
+    for j in range(g.T):
+        v[0, :, j, g.scale_of[j]] = 1.0
+    O, mass = oracle.block_causal_attention(q, k, v, sides, np.array([1.5, 0.6]),
+                                            gen_bias(3, 2, g.S).astype(np.float64))
+    np.testing.assert_allclose(O, mass, atol=1e-13, rtol=0)
+
+
+def _sdpa_reference(q, k, v, allowed, tau, bias_cols):
+    """torch fp64 scaled_dot_product_attention with a float mask: bias where
+    allowed, -inf elsewhere; scale tau/sqrt(D)."""
+    D = q.shape[-1]
+    qt = torch.from_numpy(q)[None]
+    kt = torch.from_numpy(k)[None]
+    vt = torch.from_numpy(v)[None]
+    mask = torch.full(allowed.shape, float("-inf"), dtype=torch.float64)
+    mask[torch.from_numpy(allowed)] = 0.0
+    mask = mask + torch.from_numpy(bias_cols)[None, :]
+    o = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask[None],
+                                                         scale=float(tau) / math.sqrt(D))
+    return o[0].numpy()
+
+
+def test_block_causal_matches_library_attention_with_mask():
+    """Whole block-causal stack vs torch SDPA with an explicit scale mask."""
+    sides = SIDES_TINY
+    g = _geom(sides)
+    q, k, v = _qkv(1, 2, g.T, 64, tag=4)
+    tau = np.array([0.55, 1.8])
+    bias = gen_bias(4, 2, g.S).astype(np.float64)
+    O, _ = oracle.block_causal_attention(q, k, v, sides, tau, bias)
+    sc = np.array(g.scale_of)
+    allowed = sc[None, :] <= sc[:, None]
+    for h in range(2):
+        ref = _sdpa_reference(q[0, h], k[0, h], v[0, h], allowed, tau[h], bias[h][sc])
+        np.testing.assert_allclose(O[0, h], ref, atol=1e-12, rtol=0)
+
+
+def test_single_scale_is_textbook_attention():
+    sides = (5,)
+    q, k, v = _qkv(1, 1, 25, 32, tag=5)
+    O, mass = oracle.block_causal_attention(q, k, v, sides, np.array([1.25]), None)
+    ref = _sdpa_reference(q[0, 0], k[0, 0], v[0, 0], np.ones((25, 25), bool), 1.25, np.zeros(25))
+    np.testing.assert_allclose(O[0, 0], ref, atol=1e-13, rtol=0)
+    np.testing.assert_allclose(mass[..., 0], 1.0, atol=1e-14)
+
+
+def test_pruned_at_full_budget_is_full_attention_bit_exact():
+    sides = SIDES_TINY
+    g = _geom(sides)
+    q, k, v = _qkv(2, 2, g.T, 64, tag=6)
+    tau = np.array([0.9, 1.4])
+    bias = gen_bias(6, 2, g.S).astype(np.float64)
+    O_full, _ = oracle.block_causal_attention(q, k, v, sides, tau, bias)
+    keep = np.ones((2, g.S), dtype=np.uint8)
+    O_pr = oracle.pruned_attention(q, k, v, keep, sides, tau, bias)
+    assert np.array_equal(O_full, O_pr)
+
+
+def test_pruned_matches_library_attention_with_keep_mask():
+    sides = SIDES_TINY
+    g = _geom(sides)
+    q, k, v = _qkv(1, 3, g.T, 64, tag=7)
+    tau = np.array([0.9, 1.4, 0.6])
+    bias = gen_bias(7, 3, g.S).astype(np.float64)
+    rng = np.random.default_rng(7)
+    keep = rng.integers(0, 2, size=(3, g.S)).astype(np.uint8)
+    keep[:, :2] = 1
+    O = oracle.pruned_attention(q, k, v, keep, sides, tau, bias)
+    sc = np.array(g.scale_of)
+    for h in range(3):
+        allowed = ((sc[None, :] < sc[:, None]) & (keep[h][sc][None, :] == 1)) | (sc[None, :] == sc[:, None])
+        ref = _sdpa_reference(q[0, h], k[0, h], v[0, h], allowed, tau[h], bias[h][sc])
+        np.testing.assert_allclose(O[0, h], ref, atol=1e-12, rtol=0)
+    # single-query-scale form gives the same rows
+    kq = 5
+    O5 = oracle.pruned_attention(q[:, :, g.off[kq]:g.off[kq] + g.n[kq]], k, v, keep, sides, tau, bias, query_scale=kq)
+    np.testing.assert_array_equal(O5, O[:, :, g.off[kq]:g.off[kq] + g.n[kq]])
+
+
+def test_constant_values_give_constant_output():
+    sides = SIDES_TINY
+    g = _geom(sides)
+    q, k, _ = _qkv(1, 2, g.T, 64, tag=8)
+    v = np.full((1, 2, g.T, 64), 0.375)
+    O, _ = oracle.block_causal_attention(q, k, v, sides, np.array([1.0, 2.0]), None)
+    np.testing.assert_allclose(O, 0.375, atol=1e-14, rtol=0)
+    keep = np.zeros((2, g.S), dtype=np.uint8)
+    O2 = oracle.pruned_attention(q, k, v, keep, sides, np.array([1.0, 2.0]))
+    np.testing.assert_allclose(O2, 0.375, atol=1e-14, rtol=0)
+
+
+def test_row_helpers_agree_with_whole_stack():
+    sides = SIDES_TINY
+    g = _geom(sides)
+    q, k, v = _qkv(1, 2, g.T, 64, tag=9)
+    tau = np.array([0.8, 1.1])
+    bias = gen_bias(9, 2, g.S).astype(np.float64)
+    O, mass = oracle.block_causal_attention(q, k, v, sides, tau, bias)
+    kk = 6
+    r0, r1 = g.off[kk], g.L[kk]
+    o, m = oracle.attention_rows(q[0, 1, r0:r1], k[0, 1], v[0, 1], sides, kk, tau[1], bias[1])
+    np.testing.assert_array_equal(o, O[0, 1, r0:r1])
+    np.testing.assert_array_equal(m, mass[0, 1, r0:r1])
+    keep = np.array([1, 1, 0, 1, 0, 0, 1], dtype=np.uint8)
+    Op = oracle.pruned_attention(q, k, v, np.stack([keep, keep]), sides, tau, bias)
+    o2 = oatt.pruned_attention_rows(q[0, 0, r0:r1], k[0, 0], v[0, 0], keep, sides, kk, tau[0], bias[0])
+    np.testing.assert_array_equal(o2, Op[0, 0, r0:r1])
+
+
+# ---------------------------------------------------------------- schedule
+
+def _brute_force_drop_set(scores, sizes, budget_bp, F, base_kept):
+    """Smallest rank-closed feasible drop set, by enumeration of all subsets.
+    Rank-closed: every candidate ranked below a dropped one is dropped too,
+    ranks compared pairwise on (score, index)."""
+    n = len(scores)
+    keys = [(scores[i], i) for i in range(n)]
+    best = None
+    for mask in range(1 << n):
+        X = [i for i in range(n) if mask >> i & 1]
+        closed = all(keys[y] > keys[x] for x in X for y in range(n) if not (mask >> y & 1))
+        if not closed:
+            continue
+        kept = base_kept - sum(sizes[i] for i in X)
+        if kept * 10000 > budget_bp * F:
+            continue
+        if best is None or len(X) < len(best):
+            best = X
+    return best
+
+
+@pytest.mark.parametrize("trial", range(6))
+def test_schedule_matches_brute_force_on_eight_pairs(trial):
+    sides = (1, 2, 3, 4, 5, 6)          # 4 candidates per head with sinks 0-1
+    g = _geom(sides)
+    L, H, n_sinks = 1, 2, 2
+    rng = np.random.default_rng(100 + trial)
+    scas = rng.uniform(0, 1, size=(L, H, g.S))
+    if trial % 2:
+        scas = np.round(scas, 1)            # force ties -> index tie-break
+    cand = [(l, h, s) for l in range(L) for h in range(H) for s in range(n_sinks, g.S)]
+    assert len(cand) == 8
+    F = L * H * g.T
+    for budget in range(0, 10001, 250):
+        sink = L * H * sum(g.n[:n_sinks])
+        if sink * 10000 > budget * F:
+            with pytest.raises(oracle.BudgetError):
+                oracle.build_schedule(scas, sides, budget, n_sinks)
+            continue
+        keep = oracle.build_schedule(scas, sides, budget, n_sinks)
+        dropped = [i for i, (l, h, s) in enumerate(cand) if keep[l, h, s] == 0]
+        # the ranking key uses the position in index order as the tie-break
+        bf = _brute_force_drop_set([scas[c] for c in cand], [g.n[c[2]] for c in cand], budget, F, F)
+        assert sorted(dropped) == sorted(bf), (budget, dropped, bf)
+        assert np.all(keep[:, :, :n_sinks] == 1)
+        kept = int((keep * np.array(g.n)[None, None, :]).sum())
+        assert kept * 10000 <= budget * F
+
+
+def test_schedule_special_cases():
+    sides = SIDES_TINY
+    g = _geom(sides)
+    scas = np.random.default_rng(0).uniform(size=(2, 3, g.S))
+    assert np.all(oracle.build_schedule(scas, sides, 10000, 2) == 1)
+    # all-zero S-CAS: drop order is plain index order (l, h, s)
+    keep = oracle.build_schedule(np.zeros((2, 3, g.S)), sides, 9000, 2)
+    F = 2 * 3 * g.T
+    order = [(l, h, s) for l in range(2) for h in range(3) for s in range(2, g.S)]
+    kept, ndrop = F, 0
+    while kept * 10000 > 9000 * F:
+        kept -= g.n[order[ndrop][2]]
+        ndrop += 1
+    for i, (l, h, s) in enumerate(order):
+        assert keep[l, h, s] == (0 if i < ndrop else 1)
+    with pytest.raises(oracle.BudgetError):
+        oracle.build_schedule(scas, sides, 10, 2)       # 0.1% < sinks (5/155)
+    # the last scale scores 0 and is dropped first
+    scas2 = np.random.default_rng(1).uniform(0.1, 1, size=(1, 2, g.S))
+    scas2[:, :, -1] = 0.0
+    keep2 = oracle.build_schedule(scas2, sides, 7000, 2)
+    assert np.all(keep2[0, :, -1] == 0)
+
+
+# ---------------------------------------------------------------- layout
+
+def test_offsets_closed_form_all_kept():
+    sides = SIDES_TINY
+    g = _geom(sides)
+    L, H, B, D = 3, 4, 2, 64
+    keep = np.ones((L, H, g.S), dtype=np.uint8)
+    head_off, seg_off, past_len, layer_base = oracle.build_offsets(keep, sides, B, D)
+    for l in range(L):
+        for h in range(H):
+            assert head_off[l, h] == h * g.T
+            for s in range(g.S):
+                assert seg_off[l, h, s] == g.off[s]
+                assert past_len[l, h, s] == g.off[s]
+    assert list(layer_base) == [l * B * H * g.T * D for l in range(L + 1)]
+
+
+def test_offsets_invariants_random_keep():
+    sides = SIDES_TINY
+    g = _geom(sides)
+    L, H, B, D = 2, 5, 3, 64
+    keep = np.random.default_rng(5).integers(0, 2, size=(L, H, g.S)).astype(np.uint8)
+    head_off, seg_off, past_len, layer_base = oracle.build_offsets(keep, sides, B, D)
+    for l in range(L):
+        R = [sum(g.n[s] for s in range(g.S) if keep[l, h, s]) for h in range(H)]
+        assert list(head_off[l]) == [sum(R[:h]) for h in range(H)]
+        assert layer_base[l + 1] - layer_base[l] == B * sum(R) * D
+        for h in range(H):
+            prev_end = 0
+            for s in range(g.S):
+                assert past_len[l, h, s] == sum(g.n[t] for t in range(s) if keep[l, h, t])
+                if keep[l, h, s]:
+                    assert seg_off[l, h, s] == prev_end
+                    prev_end += g.n[s]
+                else:
+                    assert seg_off[l, h, s] == -1
+
+
+def test_compaction_identity_coded():
+    """Source words encode their (l, b, h, t, d); every destination word must
+    decode to a token of a kept scale, each exactly once, in (h, s, raster) order."""
+    sides = SIDES_TINY
+    g = _geom(sides)
+    L, B, H, D = 2, 2, 3, 8
+    T = g.T
+    ids = np.arange(L * B * H * T, dtype=np.int64).reshape(L, B, H, T)
+    kd = np.zeros((L, B, H, T, D), dtype=np.uint16)
+    vd = np.zeros((L, B, H, T, D), dtype=np.uint16)
+    for d in range(D):
+        kd[..., d] = (ids * 8 + d) & 0xFFFF          # 1860 rows * 8 < 65536
+        vd[..., d] = (0xFFFF - (ids * 8 + d)) & 0xFFFF
+    keep = np.random.default_rng(11).integers(0, 2, size=(L, H, g.S)).astype(np.uint8)
+    head_off, seg_off, past_len, layer_base = oracle.build_offsets(keep, sides, B, D)
+    kc, vc = oracle.compact_kv(kd, vd, keep, sides, head_off, seg_off, layer_base)
+    assert np.array_equal(vc, (0xFFFF - kc.astype(np.int64)).astype(np.uint16))
+    rows = kc.reshape(-1, D)
+    assert np.all(rows[:, 1:] - rows[:, :1] == np.arange(1, D, dtype=np.uint16)[None, :])
+    decoded = rows[:, 0].astype(np.int64) // 8
+    pos = 0
+    for l in range(L):
+        for b in range(B):
+            for h in range(H):
+                for s in range(g.S):
+                    if keep[l, h, s]:
+                        for t in range(g.off[s], g.off[s] + g.n[s]):
+                            lb, bb, hh, tt = np.unravel_index(decoded[pos], (L, B, H, T))
+                            assert (lb, bb, hh, tt) == (l, b, h, t)
+                            pos += 1
+    assert pos == rows.shape[0]
+
+
+# ---------------------------------------------------------------- planted mistakes
+
+def _mutant_checks(monkeypatch, patch):
+    """Apply a planted mistake to the oracle and report which pins fail."""
+    patch(monkeypatch)
+    failures = 0
+    for fn in (test_mass_rows_sum_to_one_and_scas_column_sums, test_bias_only_closed_form,
+               test_block_causal_matches_library_attention_with_mask,
+               test_pruned_matches_library_attention_with_keep_mask,
+               test_scale_indicator_values_reproduce_mass):
+        try:
+            fn()
+        except AssertionError:
+            failures += 1
+    return failures
+
+
+def _patch_no_tau(mp):
+    orig = oatt.attend
+    mp.setattr(oatt, "attend", lambda q, k, v, tau, cb, D: orig(q, k, v, 1.0, cb, D))
+
+
+def _patch_bias_sign(mp):
+    orig = oatt.attend
+    mp.setattr(oatt, "attend", lambda q, k, v, tau, cb, D: orig(q, k, v, tau, -cb, D))
+
+
+def _patch_mask_off_by_one(mp):
+    G = oatt.ScaleGeometry
+
+    class Shifted(G):
+        def __init__(self, sides):
+            super().__init__(sides)
+            self.L = [self.L[min(k + 1, self.S - 1)] for k in range(self.S)]
+    mp.setattr(oatt, "ScaleGeometry", Shifted)
+
+
+def _patch_transposed_scale(mp):
+    orig = oatt._col_bias
+    mp.setattr(oatt, "_col_bias", lambda g, b, ks: orig(g, b, list(reversed(list(ks)))))
+
+
+@pytest.mark.parametrize("patch", [_patch_no_tau, _patch_bias_sign, _patch_mask_off_by_one,
+                                   _patch_transposed_scale])
+def test_planted_mistakes_are_caught(monkeypatch, patch):
+    assert _mutant_checks(monkeypatch, patch) >= 1
