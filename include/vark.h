@@ -1,0 +1,211 @@
+/*
+ * vark.h -- C ABI of the head-scale KV-cache pruning library for next-scale
+ * (VAR) transformers (HeatKV-style), B200 / sm_100a.
+ *
+ * Sources, cited by page title and section:
+ *   [HeatKV] "HeatKV: Head-tuned KV-cache Compression for Visual
+ *            Autoregressive Modeling" project page: Abstract; Method steps
+ *            1-5 (calibration prompts, per-(layer, head, source scale, future
+ *            scale) attention aggregation, S-CAS ranking, budget allocation
+ *            with retained sink scales, static schedule at inference);
+ *            Table 1 (budgets as fractions of the full cache).
+ *   [Review] machine review page of the HeatKV paper (arXiv 2605.14877):
+ *            Figure 3 caption (tokens of a scale in raster order), Figure 4
+ *            caption (Algorithm 1, BINARY-HEATKV with GREEDYEARLYPRUNING).
+ *   [AMS-KV] "AMS-KV: Adaptive KV Caching in Multi-Scale Visual
+ *            Autoregressive Transformers" listing: Abstract (attending to the
+ *            local scale matters most; condensed early scales).
+ *
+ * Conventions shared by every call
+ *   - bf16 tensors are passed as `const uint16_t*` holding raw bf16 bits.
+ *   - "dev" pointers are CUDA device pointers, "host" pointers host memory.
+ *     The caller owns all memory; the library allocates nothing, keeps no
+ *     state between calls and is safe to call from several host threads.
+ *   - Device calls are asynchronous on `stream` (a cudaStream_t passed as
+ *     void*; NULL = the legacy default stream).  Host calls are synchronous.
+ *   - Every call returns a status: VARK_OK (0) or a negative VARK_E_* code.
+ *     On an argument error nothing is launched and no output is touched.
+ *   - Device pointers and row strides must be 16-byte aligned (VARK_E_ALIGN).
+ *   - Scale lists: `sides[S]` (host) gives the side of each square token map,
+ *     ascending; scale s holds n_s = sides[s]^2 tokens, token maps are stored
+ *     scale after scale, raster order inside a scale, so
+ *     off_s = sum_{s'<s} n_s', T = sum_s n_s.  1 <= S <= VARK_MAX_SCALES.
+ *   - Logit of query i and key j of head h:
+ *       x_ij = tau[h] * (q_i . k_j) / sqrt(D) + bias[h][scale(j)]
+ *     (bias may be NULL = 0).  Softmax over the keys a query sees; fp32
+ *     accumulation on bf16 inputs; outputs rounded to bf16 (RNE).
+ *
+ * Memory layout of the compacted (pruned) cache, defined by this library:
+ *   R[l][h]          = sum_s keep[l][h][s] * n_s       rows kept by head h
+ *   R_l              = sum_h R[l][h]                   rows per batch element
+ *   head_off[l][h]   = sum_{h'<h} R[l][h']
+ *   seg_off[l][h][s] = sum_{s'<s} keep[l][h][s'] * n_s'  if kept, else -1
+ *   past_len[l][h][k]= sum_{s<k} keep[l][h][s] * n_s
+ *   layer_base[l]    = sum_{l'<l} B * R_l' * D           (elements, L+1 entries)
+ *   Layer l's compacted K (and V) is a [B][R_l][D] bf16 block at element
+ *   layer_base[l]; token t of kept scale s of (b, h) is row
+ *   b*R_l + head_off[l][h] + seg_off[l][h][s] + t of that block.
+ */
+#ifndef VARK_H
+#define VARK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define VARK_MAX_SCALES 32
+
+enum vark_status {
+  VARK_OK = 0,
+  VARK_E_ARG = -1,      /* null pointer, negative size or otherwise bad argument */
+  VARK_E_SHAPE = -2,    /* unsupported shape (e.g. D not 64/128, S out of range, size overflow) */
+  VARK_E_ALIGN = -3,    /* pointer or stride not 16-byte aligned */
+  VARK_E_BUDGET = -4,   /* the sink scales alone exceed the requested budget */
+  VARK_E_CUDA = -5,     /* a CUDA runtime / driver call failed (launch, tensor map) */
+  VARK_E_TIMEOUT = -6,  /* a bounded device wait gave up; written to *dev_status */
+  VARK_E_DEVICE = -7    /* the current device is not an sm_100 part */
+};
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* vark_status_string(int status);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int vark_version(void);
+
+/*
+ * vark_scas_accumulate -- S-CAS calibration attention of one layer.
+ * [HeatKV] Method step 2: attention probabilities aggregated for each layer,
+ * head, source scale and future (query) scale.
+ *
+ * Block-causal multi-scale attention: a query of scale k attends to every key
+ * of scales 0..k (its own scale included, [Review] Figure 3 caption).  For
+ * every query row i of scale k and source scale s <= k the probability mass
+ * m_i(s) = sum_{j in scale s} p_ij is reduced over the B * n_k rows of scale k
+ * and their MEAN is ADDED to mass[h][s][k]:
+ *     mass[h][s][k] += (1 / (B * n_k)) * sum_{b, i in scale k} m_i(s)
+ * With calibration seeds folded into the batch one call already averages the
+ * seeds; several calls accumulate (divide by the call count when finalising).
+ *
+ *   q, k, v    dev  bf16 [B][H][T][D], contiguous.
+ *   B, H       batch (calibration seeds) and heads, >= 1.
+ *   D          head dimension, 64 or 128.
+ *   S, sides   host scale list (see conventions).
+ *   tau        dev  fp32 [H] per-head temperature.
+ *   bias       dev  fp32 [H][S] additive logit bias per source scale, or NULL.
+ *   mass       dev  fp32 [H][S][S], indexed [h][s][k]; accumulated with fp32
+ *              atomics (one per (h, s, k) per CTA): entries s > k untouched.
+ *   out        dev  bf16 [B][H][T][D] attention output O, or NULL to skip it.
+ *   dev_status dev  int32, required; the caller sets it to 0 before the call;
+ *              a kernel that gives up a bounded wait stores VARK_E_TIMEOUT.
+ * Errors: VARK_E_ARG, VARK_E_SHAPE, VARK_E_ALIGN, VARK_E_CUDA, VARK_E_DEVICE.
+ */
+int vark_scas_accumulate(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                         int B, int H, int D, int S, const int32_t* sides,
+                         const float* tau, const float* bias,
+                         float* mass, uint16_t* out, int32_t* dev_status, void* stream);
+
+/*
+ * vark_scas_finalize -- host.  [HeatKV] Abstract / Method step 3: the
+ * Scale-dependent Cumulative Attention Score of a (layer, head, source scale):
+ *     scas[l][h][s] = (1 / n_calls) * sum_{k > s} mass[l][h][s][k]
+ * i.e. the attention mass a head puts on scale s, summed over the future scales
+ * that read it (the last scale scores 0).
+ *   mass  host fp32 [L][H][S][S] as accumulated by vark_scas_accumulate
+ *         (one [H][S][S] block per layer) over n_calls calls per layer.
+ *   scas  host fp64 [L][H][S] output.
+ * Errors: VARK_E_ARG (null, n_calls < 1), VARK_E_SHAPE.
+ */
+int vark_scas_finalize(const float* mass, int L, int H, int S, int n_calls, double* scas);
+
+/*
+ * vark_build_schedule -- host.  [HeatKV] Method steps 3-4 and Abstract: remove
+ * the lowest-ranked head-scale pairs until a user-selected memory budget is met,
+ * always retaining the early sink scales; one static schedule per budget.
+ *
+ *   F = L * H * T tokens (the whole cache at the end of generation).
+ *   Candidates: every (l, h, s) with s >= n_sinks, in ascending order of
+ *   (scas[l][h][s], l, h, s) -- ties broken by index.  Pairs are dropped in
+ *   that order until kept * 10000 <= budget_bp * F (the first point where the
+ *   budget holds; equality meets it).  The local scale of a query is attended
+ *   from the dense cache at inference, so it is not exempt here.
+ *
+ *   scas       host fp64 [L][H][S] (finite).
+ *   budget_bp  budget in basis points of F, 0..10000 (10000 keeps everything).
+ *   n_sinks    number of leading sink scales never dropped, 0..S.
+ *   keep       host uint8 [L][H][S] output, 1 = retained.
+ * Errors: VARK_E_ARG (null, non-finite scas, budget > 10000), VARK_E_SHAPE,
+ *         VARK_E_BUDGET (the sinks alone exceed the budget; keep untouched).
+ */
+int vark_build_schedule(const double* scas, int L, int H, int S, const int32_t* sides,
+                        uint32_t budget_bp, int n_sinks, uint8_t* keep);
+
+/*
+ * vark_build_offsets -- device.  Offset tables of the ragged per-head layout
+ * (see the layout block above) from a keep schedule.
+ *   keep        dev uint8 [L][H][S] (0 / non-zero).
+ *   B, D        batch and head dimension used for layer_base.
+ *   head_off    dev int32 [L][H]      out
+ *   seg_off     dev int32 [L][H][S]   out (-1 for dropped scales)
+ *   past_len    dev int32 [L][H][S]   out
+ *   layer_base  dev int64 [L + 1]     out (elements; layer_base[L] = total)
+ * Limits: L * H <= 16384, every R_l * B fits in int32.
+ * Errors: VARK_E_ARG, VARK_E_SHAPE, VARK_E_ALIGN, VARK_E_CUDA.
+ */
+int vark_build_offsets(const uint8_t* keep, int L, int H, int S, const int32_t* sides, int B, int D,
+                       int32_t* head_off, int32_t* seg_off, int32_t* past_len, int64_t* layer_base,
+                       void* stream);
+
+/*
+ * vark_compact_kv -- device.  Applies a keep schedule ([HeatKV] Method step 5):
+ * for every (l, b, h, s) with keep[l][h][s] the K and V rows [off_s, off_s+n_s)
+ * of (l, b, h) are copied, bit for bit, to their place in the compacted layout.
+ * Dropped scales are not read.  One launch covers all layers.
+ *   k, v         dev bf16, layer l's dense cache is the [B][H][T][D] block at
+ *                element l * layer_stride (layer_stride >= B*H*T*D).
+ *   keep, head_off, seg_off, layer_base   dev tables from vark_build_offsets.
+ *   kc, vc       dev bf16 outputs of layer_base[L] elements each.
+ * Errors: VARK_E_ARG, VARK_E_SHAPE (D % 8 != 0), VARK_E_ALIGN, VARK_E_CUDA.
+ */
+int vark_compact_kv(const uint16_t* k, const uint16_t* v, int64_t layer_stride,
+                    int L, int B, int H, int S, int D, const int32_t* sides,
+                    const uint8_t* keep, const int32_t* head_off, const int32_t* seg_off,
+                    const int64_t* layer_base, uint16_t* kc, uint16_t* vc, void* stream);
+
+/*
+ * vark_pruned_attention -- device.  Pruned-cache attention of one layer
+ * ([HeatKV] Method step 5 with the head-specific schedule of the Abstract;
+ * [AMS-KV] Abstract: the local scale is always attended).  A query of scale k
+ * of head h attends to that head's retained past scales s < k (ascending,
+ * read from the compacted cache: past_len[h][k] rows starting at row
+ * b*R_l + head_off[h]) followed by all n_k rows of its own scale k (read from
+ * the dense cache).  Online-softmax attention, fp32 accumulation.
+ *
+ *   q            dev bf16 queries: [B][H][T][D] when query_scale = -1 (every
+ *                scale), or [B][H][n_k][D] for query_scale = k.
+ *   kc, vc       dev bf16 this layer's compacted block, [B][R_l][D] with
+ *                kc_rows = B * R_l rows (kc, vc point at layer_base[l]).
+ *   k_dense, v_dense  dev bf16 [B][H][T][D] this layer's dense cache (only
+ *                the local-scale rows are read).
+ *   head_off     dev int32 [H]     this layer's row of the offset tables
+ *   seg_off      dev int32 [H][S]  (used for the bias of compacted keys)
+ *   past_len     dev int32 [H][S]
+ *   tau, bias    dev fp32 [H] and [H][S] (bias may be NULL).
+ *   out          dev bf16, same shape as q.
+ *   dev_status   dev int32, required (see vark_scas_accumulate).
+ * Errors: VARK_E_ARG, VARK_E_SHAPE, VARK_E_ALIGN, VARK_E_CUDA, VARK_E_DEVICE.
+ */
+int vark_pruned_attention(const uint16_t* q, const uint16_t* kc, const uint16_t* vc, int64_t kc_rows,
+                          const uint16_t* k_dense, const uint16_t* v_dense,
+                          int B, int H, int S, int D, const int32_t* sides, int query_scale,
+                          const int32_t* head_off, const int32_t* seg_off, const int32_t* past_len,
+                          const float* tau, const float* bias,
+                          uint16_t* out, int32_t* dev_status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VARK_H */

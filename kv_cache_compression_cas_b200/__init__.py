@@ -1,0 +1,202 @@
+"""Python binding of the vark C ABI (include/vark.h): head-scale KV-cache
+pruning for next-scale (VAR) transformers on B200.
+
+Argument marshalling only -- every step of the path runs in the CUDA library
+`libvark.so` built in-tree from `csrc/` (see `build.py`).  Functions carry the
+C names; torch tensors supply device memory, `torch.cuda.current_stream()`
+the stream.  A missing library raises at first use; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libvark.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "vark.h")
+
+VARK_OK = 0
+STATUS_NAMES = {0: "VARK_OK", -1: "VARK_E_ARG", -2: "VARK_E_SHAPE", -3: "VARK_E_ALIGN", -4: "VARK_E_BUDGET",
+                -5: "VARK_E_CUDA", -6: "VARK_E_TIMEOUT", -7: "VARK_E_DEVICE"}
+
+_lib = None
+
+
+class VarkError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        super().__init__(f"{where}: {STATUS_NAMES.get(self.status, self.status)} "
+                         f"({_load().vark_status_string(self.status).decode()})")
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_I64 = ctypes.c_int64
+_U32 = ctypes.c_uint32
+
+_SIGNATURES = {
+    "vark_status_string": (ctypes.c_char_p, [_I]),
+    "vark_version": (_I, []),
+    "vark_scas_accumulate": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
+    "vark_scas_finalize": (_I, [_P, _I, _I, _I, _I, _P]),
+    "vark_build_schedule": (_I, [_P, _I, _I, _I, _P, _U32, _I, _P]),
+    "vark_build_offsets": (_I, [_P, _I, _I, _I, _P, _I, _I, _P, _P, _P, _P, _P]),
+    "vark_compact_kv": (_I, [_P, _P, _I64, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "vark_pruned_attention": (_I, [_P, _P, _P, _I64, _P, _P, _I, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P, _P,
+                                   _P, _P]),
+}
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m kv_cache_compression_cas_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def library():
+    """The loaded ctypes library."""
+    return _load()
+
+
+def header_symbols():
+    """Names of the functions declared in include/vark.h."""
+    with open(HEADER_PATH) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(vark_\w+)\s*\(", text, re.M)))
+
+
+def _check(rc: int, where: str):
+    if rc != VARK_OK:
+        raise VarkError(rc, where)
+
+
+def _sides_arg(sides):
+    arr = np.ascontiguousarray(np.asarray(sides, dtype=np.int32))
+    return arr, arr.ctypes.data
+
+
+def _dptr(t, dtype=None, name="tensor"):
+    """Device pointer of a contiguous CUDA tensor (None -> NULL)."""
+    if t is None:
+        return None
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+# ------------------------------------------------------------------ C ABI calls
+def vark_status_string(status: int) -> str:
+    return _load().vark_status_string(int(status)).decode()
+
+
+def vark_version() -> int:
+    return int(_load().vark_version())
+
+
+def vark_scas_accumulate(q, k, v, sides, tau, bias, mass, out=None, dev_status=None, stream=None):
+    """S-CAS calibration attention of one layer (see vark.h).  q/k/v bf16
+    [B][H][T][D]; tau fp32 [H]; bias fp32 [H][S] or None; mass fp32 [H][S][S]
+    accumulated; out bf16 like q or None; dev_status int32 [1]."""
+    import torch
+    B, H, T, D = q.shape
+    s_arr, s_ptr = _sides_arg(sides)
+    rc = _load().vark_scas_accumulate(
+        _dptr(q, torch.bfloat16, "q"), _dptr(k, torch.bfloat16, "k"), _dptr(v, torch.bfloat16, "v"),
+        B, H, D, len(s_arr), s_ptr, _dptr(tau, torch.float32, "tau"), _dptr(bias, torch.float32, "bias"),
+        _dptr(mass, torch.float32, "mass"), _dptr(out, torch.bfloat16, "out"),
+        _dptr(dev_status, torch.int32, "dev_status"), _stream(stream))
+    _check(rc, "vark_scas_accumulate")
+
+
+def vark_scas_finalize(mass: np.ndarray, n_calls: int = 1) -> np.ndarray:
+    """Host: S-CAS [L][H][S] fp64 from accumulated mass [L][H][S][S] fp32."""
+    m = np.ascontiguousarray(mass, dtype=np.float32)
+    if m.ndim == 3:
+        m = m[None]
+    L, H, S, _ = m.shape
+    out = np.zeros((L, H, S), dtype=np.float64)
+    _check(_load().vark_scas_finalize(m.ctypes.data, L, H, S, int(n_calls), out.ctypes.data), "vark_scas_finalize")
+    return out
+
+
+def vark_build_schedule(scas: np.ndarray, sides, budget_bp: int, n_sinks: int) -> np.ndarray:
+    """Host: keep uint8 [L][H][S] for a budget in basis points."""
+    sc = np.ascontiguousarray(scas, dtype=np.float64)
+    L, H, S = sc.shape
+    s_arr, s_ptr = _sides_arg(sides)
+    keep = np.zeros((L, H, S), dtype=np.uint8)
+    _check(_load().vark_build_schedule(sc.ctypes.data, L, H, S, s_ptr, int(budget_bp), int(n_sinks),
+                                       keep.ctypes.data), "vark_build_schedule")
+    return keep
+
+
+def vark_build_offsets(keep, sides, B: int, D: int, head_off, seg_off, past_len, layer_base, stream=None):
+    """Device: offset tables into caller-provided int32/int64 tensors."""
+    import torch
+    L, H, S = keep.shape
+    s_arr, s_ptr = _sides_arg(sides)
+    rc = _load().vark_build_offsets(
+        _dptr(keep, torch.uint8, "keep"), L, H, S, s_ptr, int(B), int(D),
+        _dptr(head_off, torch.int32, "head_off"), _dptr(seg_off, torch.int32, "seg_off"),
+        _dptr(past_len, torch.int32, "past_len"), _dptr(layer_base, torch.int64, "layer_base"), _stream(stream))
+    _check(rc, "vark_build_offsets")
+
+
+def vark_compact_kv(k, v, layer_stride: int, L: int, B: int, H: int, sides, D: int, keep, head_off, seg_off,
+                    layer_base, kc, vc, stream=None):
+    """Device: gather retained scale blocks of all layers into kc / vc."""
+    import torch
+    s_arr, s_ptr = _sides_arg(sides)
+    rc = _load().vark_compact_kv(
+        _dptr(k, torch.bfloat16, "k"), _dptr(v, torch.bfloat16, "v"), int(layer_stride), int(L), int(B), int(H),
+        len(s_arr), int(D), s_ptr, _dptr(keep, torch.uint8, "keep"), _dptr(head_off, torch.int32, "head_off"),
+        _dptr(seg_off, torch.int32, "seg_off"), _dptr(layer_base, torch.int64, "layer_base"),
+        _dptr(kc, torch.bfloat16, "kc"), _dptr(vc, torch.bfloat16, "vc"), _stream(stream))
+    _check(rc, "vark_compact_kv")
+
+
+def vark_pruned_attention(q, kc, vc, kc_rows: int, k_dense, v_dense, sides, query_scale: int, head_off, seg_off,
+                          past_len, tau, bias, out, dev_status, stream=None):
+    """Device: pruned-cache attention of one layer (see vark.h)."""
+    import torch
+    B, H = k_dense.shape[0], k_dense.shape[1]
+    D = k_dense.shape[3]
+    s_arr, s_ptr = _sides_arg(sides)
+    kcp = kc.data_ptr() if (kc is not None and kc_rows > 0) else None
+    vcp = vc.data_ptr() if (vc is not None and kc_rows > 0) else None
+    if kc is not None:
+        _dptr(kc, torch.bfloat16, "kc")
+        _dptr(vc, torch.bfloat16, "vc")
+    rc = _load().vark_pruned_attention(
+        _dptr(q, torch.bfloat16, "q"), kcp, vcp, int(kc_rows),
+        _dptr(k_dense, torch.bfloat16, "k_dense"), _dptr(v_dense, torch.bfloat16, "v_dense"),
+        int(B), int(H), len(s_arr), int(D), s_ptr, int(query_scale),
+        _dptr(head_off, torch.int32, "head_off"), _dptr(seg_off, torch.int32, "seg_off"),
+        _dptr(past_len, torch.int32, "past_len"), _dptr(tau, torch.float32, "tau"),
+        _dptr(bias, torch.float32, "bias"), _dptr(out, torch.bfloat16, "out"),
+        _dptr(dev_status, torch.int32, "dev_status"), _stream(stream))
+    _check(rc, "vark_pruned_attention")

@@ -1,0 +1,112 @@
+// Host-only exports: status strings, S-CAS finalisation and the static
+// keep-schedule builder.
+//
+// [HeatKV] project page, Abstract and Method steps 3-4: head-scale pairs are
+// ranked by S-CAS and the lowest-ranked are removed until the user's memory
+// budget holds, the early sink scales always retained; the schedule is built
+// once, offline, before inference.
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <vector>
+
+#include "vark.h"
+
+extern "C" const char* vark_status_string(int status) {
+  switch (status) {
+    case VARK_OK: return "VARK_OK";
+    case VARK_E_ARG: return "VARK_E_ARG: invalid argument";
+    case VARK_E_SHAPE: return "VARK_E_SHAPE: unsupported shape";
+    case VARK_E_ALIGN: return "VARK_E_ALIGN: pointer or stride not 16-byte aligned";
+    case VARK_E_BUDGET: return "VARK_E_BUDGET: sink scales alone exceed the budget";
+    case VARK_E_CUDA: return "VARK_E_CUDA: CUDA call failed";
+    case VARK_E_TIMEOUT: return "VARK_E_TIMEOUT: a bounded device wait gave up";
+    case VARK_E_DEVICE: return "VARK_E_DEVICE: current device is not sm_100";
+    default: return "VARK: unknown status";
+  }
+}
+
+extern "C" int vark_version(void) { return 10000; }
+
+static bool sides_ok(int S, const int32_t* sides, int64_t* T_out) {
+  if (S < 1 || S > VARK_MAX_SCALES || sides == nullptr) return false;
+  int64_t T = 0;
+  for (int s = 0; s < S; ++s) {
+    if (sides[s] < 1 || sides[s] > 4096) return false;
+    T += int64_t(sides[s]) * sides[s];
+  }
+  if (T > (int64_t(1) << 30)) return false;
+  *T_out = T;
+  return true;
+}
+
+extern "C" int vark_scas_finalize(const float* mass, int L, int H, int S, int n_calls, double* scas) {
+  if (mass == nullptr || scas == nullptr || n_calls < 1) return VARK_E_ARG;
+  if (L < 1 || H < 1 || S < 1 || S > VARK_MAX_SCALES) return VARK_E_SHAPE;
+  const double inv = 1.0 / double(n_calls);
+  for (int64_t lh = 0; lh < int64_t(L) * H; ++lh) {
+    const float* M = mass + lh * S * S;           // [s][k]
+    for (int s = 0; s < S; ++s) {
+      double acc = 0.0;
+      for (int k = s + 1; k < S; ++k) acc += double(M[s * S + k]);
+      scas[lh * S + s] = acc * inv;
+    }
+  }
+  return VARK_OK;
+}
+
+namespace {
+struct Candidate {
+  double score;
+  int32_t l, h, s;
+};
+}  // namespace
+
+extern "C" int vark_build_schedule(const double* scas, int L, int H, int S, const int32_t* sides,
+                                   uint32_t budget_bp, int n_sinks, uint8_t* keep) {
+  if (scas == nullptr || keep == nullptr || sides == nullptr) return VARK_E_ARG;
+  if (budget_bp > 10000u || n_sinks < 0) return VARK_E_ARG;
+  int64_t T = 0;
+  if (L < 1 || H < 1 || !sides_ok(S, sides, &T) || n_sinks > S) return VARK_E_SHAPE;
+  if (int64_t(L) * H > (int64_t(1) << 24)) return VARK_E_SHAPE;
+  const int64_t LHS = int64_t(L) * H * S;
+  for (int64_t i = 0; i < LHS; ++i)
+    if (!std::isfinite(scas[i])) return VARK_E_ARG;
+
+  std::vector<int64_t> n(S);
+  int64_t sink_per_head = 0;
+  for (int s = 0; s < S; ++s) {
+    n[s] = int64_t(sides[s]) * sides[s];
+    if (s < n_sinks) sink_per_head += n[s];
+  }
+  const int64_t F = int64_t(L) * H * T;               // full cache, tokens
+  const int64_t budget = int64_t(budget_bp);
+  int64_t kept = F;
+  if (kept * 10000 <= budget * F) {
+    std::memset(keep, 1, size_t(LHS));
+    return VARK_OK;
+  }
+  if (int64_t(L) * H * sink_per_head * 10000 > budget * F) return VARK_E_BUDGET;
+
+  std::vector<Candidate> cand;
+  cand.reserve(size_t(int64_t(L) * H * (S - n_sinks)));
+  for (int l = 0; l < L; ++l)
+    for (int h = 0; h < H; ++h)
+      for (int s = n_sinks; s < S; ++s)
+        cand.push_back({scas[(int64_t(l) * H + h) * S + s], l, h, s});
+  // Ascending (score, l, h, s): the index tie-break makes the order total.
+  std::sort(cand.begin(), cand.end(), [](const Candidate& a, const Candidate& b) {
+    if (a.score != b.score) return a.score < b.score;
+    if (a.l != b.l) return a.l < b.l;
+    if (a.h != b.h) return a.h < b.h;
+    return a.s < b.s;
+  });
+  std::memset(keep, 1, size_t(LHS));
+  for (const Candidate& c : cand) {
+    keep[(int64_t(c.l) * H + c.h) * S + c.s] = 0;
+    kept -= n[c.s];
+    if (kept * 10000 <= budget * F) break;
+  }
+  return VARK_OK;
+}

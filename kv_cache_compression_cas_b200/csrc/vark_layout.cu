@@ -1,0 +1,253 @@
+// Offset tables and cache compaction: apply a static keep[layer][head][scale]
+// schedule by gathering the retained scale blocks of every (layer, batch,
+// head) into the per-head ragged layout documented in vark.h.
+// [HeatKV] project page, Method step 5: the static schedule is applied while
+// scales are generated; the Abstract: allocation is head-specific.
+//
+// Compaction is a pure HBM stream (every retained byte read once and written
+// once, dropped bytes never touched).  Work unit = (layer, head, kept chunk of
+// <= kChunkRows rows of one scale, batch); one persistent grid walks the units.
+// Each CTA first builds, in shared memory, the prefix of kept chunks over
+// (layer, head) for its layer group, so a unit is found by one binary search
+// and a walk over at most S scales.  Copies are 16-byte vectors, coalesced,
+// with several loads in flight per thread before the stores.
+#include <algorithm>
+
+#include "vark_common.cuh"
+
+namespace vark {
+
+// ---------------------------------------------------------------- offsets
+struct OffsetsParams {
+  ScaleTable sc;
+  int L, H, B, D;
+};
+
+// One CTA.  head_off holds R[l][h] until the per-layer scan rewrites it, and
+// layer_base[l+1] holds R_l until the layer scan; global writes are visible to
+// the block after __syncthreads.
+__global__ void __launch_bounds__(1024) offsets_kernel(const uint8_t* __restrict__ keep, OffsetsParams p,
+                                                       int32_t* head_off, int32_t* seg_off, int32_t* past_len,
+                                                       int64_t* layer_base) {
+  const int LH = p.L * p.H;
+  const int S = p.sc.S;
+  for (int i = threadIdx.x; i < LH; i += blockDim.x) {
+    int32_t running = 0;
+    for (int s = 0; s < S; ++s) {
+      past_len[i * S + s] = running;
+      if (keep[i * S + s]) {
+        seg_off[i * S + s] = running;
+        running += p.sc.n[s];
+      } else {
+        seg_off[i * S + s] = -1;
+      }
+    }
+    head_off[i] = running;
+  }
+  __syncthreads();
+  for (int l = threadIdx.x; l < p.L; l += blockDim.x) {
+    int64_t acc = 0;
+    for (int h = 0; h < p.H; ++h) {
+      const int32_t r = head_off[l * p.H + h];
+      head_off[l * p.H + h] = int32_t(acc);
+      acc += r;
+    }
+    layer_base[l + 1] = acc;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int64_t base = 0;
+    layer_base[0] = 0;
+    for (int l = 0; l < p.L; ++l) {
+      const int64_t rows = layer_base[l + 1];
+      base += rows * p.B * p.D;
+      layer_base[l + 1] = base;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- compaction
+constexpr int kChunkRows = 64;
+constexpr int kCompactThreads = 256;
+constexpr int kMaxGroupLH = 4096;   // (layer, head) pairs per launch group
+
+struct CompactParams {
+  ScaleTable sc;
+  int32_t chunks[VARK_MAX_SCALES];  // ceil(n_s / kChunkRows)
+  int l0, nl;                       // layer group [l0, l0 + nl)
+  int L, B, H, D;
+  int64_t layer_stride;             // elements between dense layers
+};
+
+__global__ void __launch_bounds__(kCompactThreads) compact_kernel(
+    const uint4* __restrict__ k, const uint4* __restrict__ v, CompactParams p, const uint8_t* __restrict__ keep,
+    const int32_t* __restrict__ head_off, const int32_t* __restrict__ seg_off, const int64_t* __restrict__ layer_base,
+    uint4* __restrict__ kc, uint4* __restrict__ vc) {
+  __shared__ int32_t chunk_prefix[kMaxGroupLH + 1];
+  __shared__ uint32_t keep_mask[kMaxGroupLH];
+  __shared__ int32_t warp_tot[kCompactThreads / 32];
+
+  const int S = p.sc.S;
+  const int H = p.H;
+  const int nlh = p.nl * H;
+  const int lh0 = p.l0 * H;
+
+  // 1. kept-chunk count and keep bit mask of each (layer, head) of the group
+  for (int i = threadIdx.x; i < nlh; i += kCompactThreads) {
+    const uint8_t* kp = keep + int64_t(lh0 + i) * S;
+    uint32_t m = 0;
+    int32_t c = 0;
+    for (int s = 0; s < S; ++s) {
+      if (kp[s]) {
+        m |= 1u << s;
+        c += p.chunks[s];
+      }
+    }
+    keep_mask[i] = m;
+    chunk_prefix[i] = c;
+  }
+  __syncthreads();
+  // 2. in-place exclusive scan: each thread owns a contiguous segment
+  constexpr int kPer = (kMaxGroupLH + kCompactThreads - 1) / kCompactThreads;
+  const int seg0 = threadIdx.x * kPer;
+  int32_t my_total = 0;
+  for (int u = 0; u < kPer; ++u)
+    if (seg0 + u < nlh) my_total += chunk_prefix[seg0 + u];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int32_t incl = my_total;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  int32_t warp_base = 0, grand = 0;
+#pragma unroll
+  for (int w = 0; w < kCompactThreads / 32; ++w) {
+    if (w < warp) warp_base += warp_tot[w];
+    grand += warp_tot[w];
+  }
+  int32_t run = warp_base + incl - my_total;
+  for (int u = 0; u < kPer; ++u) {
+    if (seg0 + u < nlh) {
+      const int32_t c = chunk_prefix[seg0 + u];
+      chunk_prefix[seg0 + u] = run;
+      run += c;
+    }
+  }
+  if (threadIdx.x == 0) chunk_prefix[nlh] = grand;
+  __syncthreads();
+
+  const int64_t units = int64_t(grand) * p.B;
+  const int vec_per_row = p.D / 8;  // 16-byte vectors per row
+  const int64_t T = p.sc.T;
+
+  for (int64_t g = blockIdx.x; g < units; g += gridDim.x) {
+    const int b = int(g % p.B);
+    const int32_t c = int32_t(g / p.B);
+    // (layer, head) with chunk_prefix[i] <= c < chunk_prefix[i+1]
+    int lo = 0, hi = nlh;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (chunk_prefix[mid] <= c) lo = mid; else hi = mid;
+    }
+    const int i = lo;
+    int32_t j = c - chunk_prefix[i];
+    const uint32_t m = keep_mask[i];
+    int s = 0;
+    for (; s < S; ++s) {
+      if (m >> s & 1u) {
+        if (j < p.chunks[s]) break;
+        j -= p.chunks[s];
+      }
+    }
+    const int l = p.l0 + i / H;
+    const int h = i % H;
+    const int32_t r0 = j * kChunkRows;
+    const int32_t nrows = min(kChunkRows, p.sc.n[s] - r0);
+    const int64_t R_l = (layer_base[l + 1] - layer_base[l]) / (int64_t(p.B) * p.D);
+    const int64_t dst_row = int64_t(b) * R_l + head_off[l * H + h] + seg_off[(l * H + h) * S + s] + r0;
+    const int64_t src_row = (int64_t(b) * H + h) * T + p.sc.off[s] + r0;
+    const int64_t dst_v = (layer_base[l] / 8) + dst_row * vec_per_row;
+    const int64_t src_v = (int64_t(l) * p.layer_stride) / 8 + src_row * vec_per_row;
+    const int nvec = nrows * vec_per_row;
+
+    // 4 K + 4 V vectors in flight per thread, then the stores.
+    for (int base = 0; base < nvec; base += 4 * kCompactThreads) {
+      uint4 a[4], bq[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = base + u * kCompactThreads + threadIdx.x;
+        if (e < nvec) {
+          a[u] = __ldcs(k + src_v + e);
+          bq[u] = __ldcs(v + src_v + e);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = base + u * kCompactThreads + threadIdx.x;
+        if (e < nvec) {
+          __stcs(kc + dst_v + e, a[u]);
+          __stcs(vc + dst_v + e, bq[u]);
+        }
+      }
+    }
+  }
+}
+
+}  // namespace vark
+
+using namespace vark;
+
+extern "C" int vark_build_offsets(const uint8_t* keep, int L, int H, int S, const int32_t* sides, int B, int D,
+                                  int32_t* head_off, int32_t* seg_off, int32_t* past_len, int64_t* layer_base,
+                                  void* stream) {
+  if (!keep || !head_off || !seg_off || !past_len || !layer_base) return VARK_E_ARG;
+  OffsetsParams p;
+  int rc = make_scale_table(S, sides, &p.sc);
+  if (rc) return rc;
+  if (L < 1 || H < 1 || B < 1 || D < 1) return VARK_E_SHAPE;
+  if (int64_t(L) * H > 16384) return VARK_E_SHAPE;
+  if (int64_t(B) * H * p.sc.T > INT32_MAX) return VARK_E_SHAPE;
+  if (!aligned16(head_off) || !aligned16(seg_off) || !aligned16(past_len) || !aligned16(layer_base))
+    return VARK_E_ALIGN;
+  if ((rc = check_device_sm100())) return rc;
+  p.L = L; p.H = H; p.B = B; p.D = D;
+  offsets_kernel<<<1, 1024, 0, static_cast<cudaStream_t>(stream)>>>(keep, p, head_off, seg_off, past_len, layer_base);
+  return cudaGetLastError() == cudaSuccess ? VARK_OK : VARK_E_CUDA;
+}
+
+extern "C" int vark_compact_kv(const uint16_t* k, const uint16_t* v, int64_t layer_stride, int L, int B, int H,
+                               int S, int D, const int32_t* sides, const uint8_t* keep, const int32_t* head_off,
+                               const int32_t* seg_off, const int64_t* layer_base, uint16_t* kc, uint16_t* vc,
+                               void* stream) {
+  if (!k || !v || !keep || !head_off || !seg_off || !layer_base || !kc || !vc) return VARK_E_ARG;
+  CompactParams p;
+  int rc = make_scale_table(S, sides, &p.sc);
+  if (rc) return rc;
+  if (L < 1 || H < 1 || B < 1 || D < 8 || D % 8 != 0 || D > 1024) return VARK_E_SHAPE;
+  if (H > kMaxGroupLH) return VARK_E_SHAPE;
+  if (layer_stride < int64_t(B) * H * p.sc.T * D) return VARK_E_ARG;
+  if (layer_stride % 8 != 0) return VARK_E_ALIGN;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(kc) || !aligned16(vc)) return VARK_E_ALIGN;
+  if ((rc = check_device_sm100())) return rc;
+  p.L = L; p.B = B; p.H = H; p.D = D; p.layer_stride = layer_stride;
+  for (int s = 0; s < VARK_MAX_SCALES; ++s)
+    p.chunks[s] = s < S ? (p.sc.n[s] + kChunkRows - 1) / kChunkRows : 0;
+  int dev = 0, nsm = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  const int layers_per_group = std::max(1, kMaxGroupLH / H);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  for (int l0 = 0; l0 < L; l0 += layers_per_group) {
+    p.l0 = l0;
+    p.nl = std::min(layers_per_group, L - l0);
+    compact_kernel<<<nsm * 4, kCompactThreads, 0, st>>>(reinterpret_cast<const uint4*>(k),
+                                                        reinterpret_cast<const uint4*>(v), p, keep, head_off,
+                                                        seg_off, layer_base, reinterpret_cast<uint4*>(kc),
+                                                        reinterpret_cast<uint4*>(vc));
+    if (cudaGetLastError() != cudaSuccess) return VARK_E_CUDA;
+  }
+  return VARK_OK;
+}
