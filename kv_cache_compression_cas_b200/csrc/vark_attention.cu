@@ -9,18 +9,27 @@
 //     their own scale from the dense cache.  [HeatKV] Method step 5; [AMS-KV]
 //     Abstract (the local scale is always attended).
 //
-// One CTA computes one 128-row query tile of one (batch, head) over a list of
-// 128-key tiles.  Roles (256 threads):
-//   warp 0      TMA producer: Q once, then K/V tiles into a 2-stage ring;
-//   warp 1      owns TMEM (512 columns) and issues tcgen05.mma from one thread:
-//               S_j = Q K_j^T into one of two TMEM S buffers (one tile ahead),
-//               then O += P_j V_j into the TMEM O accumulator;
-//   warps 4..7  softmax, one thread per query row (TMEM lane = row): read S_j
-//               with tcgen05.ld, online softmax in the exp2 domain, write P_j
-//               as bf16 into shared memory in the 128-byte-swizzled K-major
-//               operand layout, rescale O in TMEM only when the running max
-//               grows by more than 2^8 (the stale max cancels in O / l).
-// Operands: Q, K, P K-major SW128; V MN-major SW128 (as stored, [key][d]).
+// One CTA computes two 128-row query tiles (A, B) of the same (batch, head,
+// query scale): they see the same key list, so every K/V tile is loaded once
+// for 256 query rows.  Roles (384 threads, 3 warpgroups):
+//   warp 0       TMA producer: Q_A, Q_B, then K and V tiles into 2-stage rings
+//                with separate release points for K (after both S MMAs) and V
+//                (after both PV MMAs);
+//   warp 1       owns TMEM (512 columns) and issues tcgen05.mma from one
+//                thread, ping-ponging the tiles: PV_A(j-1), S_A(j), PV_B(j-1),
+//                S_B(j) -- so the softmax of one tile overlaps the other
+//                tile's two MMAs;
+//   warps 4-7    softmax of tile A, warps 8-11 softmax of tile B: one thread per
+//                query row (TMEM lane = row).  S_X is read with tcgen05.ld, the
+//                online softmax runs in the exp2 domain, and P_X is written back
+//                as bf16 over the first 64 columns of S_X, where the PV MMA reads
+//                it as its A operand straight from tensor memory.  O_X is
+//                rescaled in TMEM only when a row's max grows by more than 2^8
+//                (the stale max cancels in O / l).
+// TMEM: S_A [0,128) S_B [128,256) O_A [256,256+D) O_B [256+D,256+2D).
+// Shared memory: Q_A, Q_B, K and V rings, 128-byte swizzled (Q, K K-major; V
+// MN-major as stored, [key][d]).  setmaxnreg moves registers from the control
+// warpgroup to the two softmax warpgroups.
 // Every mbarrier wait is bounded: on timeout the kernel records
 // VARK_E_TIMEOUT in the caller's status word, drains its own async work with
 // bounded waits, frees TMEM and returns.
@@ -32,12 +41,12 @@
 namespace vark {
 namespace attn {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
 constexpr int kBlockM = 128;
 constexpr int kBlockN = 128;
 constexpr int kStages = 2;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kMaxQTiles = 512;
+constexpr int kMaxPairs = 512;
 constexpr int kPanelBytes = 128 * 128;   // 128 rows x 128 bytes (64 bf16)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 domain
@@ -45,8 +54,8 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 domain
 struct Params {
   ScaleTable sc;
   int B, H;
-  int n_qt;                       // query-tile kinds per (batch, head)
-  uint32_t qt[kMaxQTiles];        // (scale << 24) | row start within the scale
+  int n_pairs;                    // query-tile pairs per (batch, head)
+  uint32_t pair[kMaxPairs];       // (scale << 24) | first row of tile A within the scale
   float scale_log2;               // log2(e) / sqrt(D)
   const float* tau;
   const float* bias;              // [H][S] or null
@@ -62,34 +71,45 @@ struct Params {
   const int32_t* past_len;        // [H][S]
 };
 
+enum Bar {
+  kBarQ = 0,
+  kBarKFull = 1,      // [2]
+  kBarVFull = 3,      // [2]
+  kBarKEmpty = 5,     // [2]
+  kBarVEmpty = 7,     // [2]
+  kBarSFull = 9,      // [tile]
+  kBarPFull = 11,     // [tile]
+  kBarODone = 13,     // [tile]
+  kBarDrain = 15,
+  kNumBars = 16
+};
+
 template <int D>
 struct Smem {
   static constexpr int kQPanels = D / 64;
-  static constexpr int kQ = 0;
-  static constexpr int kK = kQ + kQPanels * kPanelBytes;
-  static constexpr int kV = kK + kStages * kQPanels * kPanelBytes;
-  static constexpr int kP = kV + kStages * kQPanels * kPanelBytes;
-  static constexpr int kMass = kP + 2 * kPanelBytes;                     // [S][128] fp32
-  static constexpr int kRed = kMass + VARK_MAX_SCALES * kBlockM * 4;     // [4][32] fp32
-  static constexpr int kBar = kRed + 4 * 32 * 4;
-  // barriers: q, k_full[2], v_full[2], kv_empty[2], s_full[2], s_free[2], p_full, o_done, drain
-  static constexpr int kNumBars = 1 + 2 * kStages + kStages + 2 + 2 + 3;
-  static constexpr int kMisc = kBar + kNumBars * 8;                       // tmem base, abort flag
-  static constexpr int kTotal = kMisc + 16;
-  static constexpr int kAlloc = kTotal + 1024;                            // alignment slack
+  static constexpr int kTile = kQPanels * kPanelBytes;
+  static constexpr int kQ = 0;                          // [2 tiles]
+  static constexpr int kK = kQ + 2 * kTile;             // [2 stages]
+  static constexpr int kV = kK + kStages * kTile;       // [2 stages]
+  static constexpr int kBar = kV + kStages * kTile;
+  static constexpr int kMisc = kBar + kNumBars * 8;     // tmem base, abort flag
+  static constexpr int kRed = kMisc + 16;               // [2 tiles][4 warps][32] fp32
+  static constexpr int kMass = kRed + 2 * 4 * 32 * 4;   // [2 tiles][S][128] fp32 (calibration)
+  static int alloc(bool mass, int S) { return kMass + (mass ? 2 * S * kBlockM * 4 : 0) + 1024; }
 };
 
-// Tile of keys j of one work item.
+// Tile j of the key list of one work item.
 struct KTile {
   int src;        // 0: dense K/V ([B*H][T][D] map), 1: compacted K/V ([rows][D] map)
   int row;        // first row (dense: within (b,h); compacted: absolute)
   int valid;      // valid key columns in this tile
-  int key0;       // first key index in the item's key list
+  int key0;       // first key index in the item's key list (segment coordinates)
 };
 
 template <bool PRUNED>
 struct Item {
-  int b, h, bh, k, qrow0, rows_valid;
+  int b, h, bh, k, row0;
+  int rows_valid[2];
   int n_tiles;
   int n_past;      // PRUNED: tiles over the compacted past
   int past;        // PRUNED: past_len[h][k]
@@ -122,17 +142,19 @@ struct Item {
 template <bool PRUNED>
 __device__ Item<PRUNED> decode_item(const Params& p) {
   Item<PRUNED> it;
-  const int BH = p.B * p.H;
-  const int kind = blockIdx.x / BH;
-  it.bh = blockIdx.x % BH;
+  // (batch, head)-major order: the CTAs in flight share a few heads' K/V in L2.
+  it.bh = blockIdx.x / p.n_pairs;
+  const int pi = blockIdx.x % p.n_pairs;
   it.b = it.bh / p.H;
   it.h = it.bh % p.H;
-  const uint32_t e = p.qt[kind];
+  const uint32_t e = p.pair[pi];
   it.k = int(e >> 24);
-  it.qrow0 = int(e & 0xFFFFFFu);
-  it.rows_valid = min(kBlockM, p.sc.n[it.k] - it.qrow0);
+  it.row0 = int(e & 0xFFFFFFu);
+  const int nk = p.sc.n[it.k];
+  it.rows_valid[0] = min(kBlockM, nk - it.row0);
+  it.rows_valid[1] = max(0, min(kBlockM, nk - it.row0 - kBlockM));
   if (!PRUNED) {
-    const int Lk = p.sc.off[it.k] + p.sc.n[it.k];
+    const int Lk = p.sc.off[it.k] + nk;
     it.n_tiles = (Lk + kBlockN - 1) / kBlockN;
     it.n_past = 0;
     it.past = 0;
@@ -140,7 +162,7 @@ __device__ Item<PRUNED> decode_item(const Params& p) {
   } else {
     it.past = p.past_len[it.h * p.sc.S + it.k];
     it.n_past = (it.past + kBlockN - 1) / kBlockN;
-    it.n_tiles = it.n_past + (p.sc.n[it.k] + kBlockN - 1) / kBlockN;
+    it.n_tiles = it.n_past + (nk + kBlockN - 1) / kBlockN;
     it.kc_row0 = int64_t(it.b) * p.R_l + p.head_off[it.h];
   }
   return it;
@@ -176,44 +198,37 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ Params p) {
   using L = Smem<D>;
   constexpr int QP = L::kQPanels;
-  constexpr uint32_t kTileBytes = QP * kPanelBytes;   // one Q / K / V tile
+  constexpr uint32_t kTileBytes = L::kTile;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t sQ = sbase + L::kQ, sK = sbase + L::kK, sV = sbase + L::kV, sP = sbase + L::kP;
-  float* mass_sm = reinterpret_cast<float*>(smem + L::kMass);
+  const uint32_t sQ = sbase + L::kQ, sK = sbase + L::kK, sV = sbase + L::kV;
   float* red_sm = reinterpret_cast<float*>(smem + L::kRed);
+  float* mass_sm = reinterpret_cast<float*>(smem + L::kMass);
   const uint32_t bar0 = sbase + L::kBar;
-  const uint32_t bar_q = bar0;
-  auto bar_k_full = [&](int s) { return bar0 + 8 * (1 + s); };
-  auto bar_v_full = [&](int s) { return bar0 + 8 * (1 + kStages + s); };
-  auto bar_kv_empty = [&](int s) { return bar0 + 8 * (1 + 2 * kStages + s); };
-  auto bar_s_full = [&](int b) { return bar0 + 8 * (1 + 3 * kStages + b); };
-  auto bar_s_free = [&](int b) { return bar0 + 8 * (3 + 3 * kStages + b); };
-  const uint32_t bar_p_full = bar0 + 8 * (5 + 3 * kStages);
-  const uint32_t bar_o_done = bar0 + 8 * (6 + 3 * kStages);
-  const uint32_t bar_drain = bar0 + 8 * (7 + 3 * kStages);
+  auto bar = [&](int i) { return bar0 + 8u * uint32_t(i); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Item<PRUNED> it = decode_item<PRUNED>(p);
   const int n = it.n_tiles;
+  const int n_act = it.rows_valid[1] > 0 ? 2 : 1;   // active query tiles
 
   if (threadIdx.x == 0) {
-    mbar_init(bar_q, 1);
+    mbar_init(bar(kBarQ), 1);
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(bar_k_full(s), 1);
-      mbar_init(bar_v_full(s), 1);
-      mbar_init(bar_kv_empty(s), 1);
+      mbar_init(bar(kBarKFull + s), 1);
+      mbar_init(bar(kBarVFull + s), 1);
+      mbar_init(bar(kBarKEmpty + s), 1);
+      mbar_init(bar(kBarVEmpty + s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(bar_s_full(b), 1);
-      mbar_init(bar_s_free(b), kBlockM);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(bar(kBarSFull + x), 1);
+      mbar_init(bar(kBarPFull + x), kBlockM);
+      mbar_init(bar(kBarODone + x), 1);
     }
-    mbar_init(bar_p_full, kBlockM);
-    mbar_init(bar_o_done, 1);
-    mbar_init(bar_drain, 1);
+    mbar_init(bar(kBarDrain), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -225,11 +240,11 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tmem_S0 = tmem, tmem_O = tmem + 256;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
+  if (warp < 4) {
+    setmaxnreg_dec56();
+    if (warp == 0 && lane == 0) {
+      // ---------------------------------------------------------- producer
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
@@ -237,144 +252,173 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         tma_prefetch_desc(&tm_kc);
         tma_prefetch_desc(&tm_vc);
       }
-      const int qrow = (p.q_scale_rows ? 0 : p.sc.off[it.k]) + it.qrow0;
-      mbar_arrive_expect_tx(bar_q, kTileBytes);
-      for (int c = 0; c < QP; ++c) tma_load_3d(sQ + c * kPanelBytes, &tm_q, bar_q, c * 64, qrow, it.bh);
-      int issued = 0;
+      const int qrow = (p.q_scale_rows ? 0 : p.sc.off[it.k]) + it.row0;
+      mbar_arrive_expect_tx(bar(kBarQ), n_act * kTileBytes);
+      for (int x = 0; x < n_act; ++x)
+        for (int c = 0; c < QP; ++c)
+          tma_load_3d(sQ + x * kTileBytes + c * kPanelBytes, &tm_q, bar(kBarQ), c * 64, qrow + x * kBlockM, it.bh);
+      int issued_k = 0, issued_v = 0;
       for (int j = 0; j < n; ++j) {
         const int st = j % kStages;
-        if (j >= kStages && !mbar_wait(bar_kv_empty(st), ((j / kStages) - 1) & 1, abort_flag, p.status)) break;
         const KTile t = it.tile(p, j);
-        mbar_arrive_expect_tx(bar_k_full(st), kTileBytes);
+        if (j >= kStages && !mbar_wait(bar(kBarKEmpty + st), ((j / kStages) - 1) & 1, abort_flag, p.status)) break;
+        mbar_arrive_expect_tx(bar(kBarKFull + st), kTileBytes);
         for (int c = 0; c < QP; ++c) {
-          const uint32_t dst = sK + (st * QP + c) * kPanelBytes;
-          if (t.src == 0) tma_load_3d(dst, &tm_k, bar_k_full(st), c * 64, t.row, it.bh);
-          else tma_load_2d(dst, &tm_kc, bar_k_full(st), c * 64, t.row);
+          const uint32_t dst = sK + st * kTileBytes + c * kPanelBytes;
+          if (t.src == 0) tma_load_3d(dst, &tm_k, bar(kBarKFull + st), c * 64, t.row, it.bh);
+          else tma_load_2d(dst, &tm_kc, bar(kBarKFull + st), c * 64, t.row);
         }
-        mbar_arrive_expect_tx(bar_v_full(st), kTileBytes);
+        issued_k = j + 1;
+        if (j >= kStages && !mbar_wait(bar(kBarVEmpty + st), ((j / kStages) - 1) & 1, abort_flag, p.status)) break;
+        mbar_arrive_expect_tx(bar(kBarVFull + st), kTileBytes);
         for (int c = 0; c < QP; ++c) {
-          const uint32_t dst = sV + (st * QP + c) * kPanelBytes;
-          if (t.src == 0) tma_load_3d(dst, &tm_v, bar_v_full(st), c * 64, t.row, it.bh);
-          else tma_load_2d(dst, &tm_vc, bar_v_full(st), c * 64, t.row);
+          const uint32_t dst = sV + st * kTileBytes + c * kPanelBytes;
+          if (t.src == 0) tma_load_3d(dst, &tm_v, bar(kBarVFull + st), c * 64, t.row, it.bh);
+          else tma_load_2d(dst, &tm_vc, bar(kBarVFull + st), c * 64, t.row);
         }
-        issued = j + 1;
+        issued_v = j + 1;
       }
-      // Drain: every load this thread issued has landed before the CTA exits
+      // Drain: every load issued here has landed before the CTA exits
       // (immediate on the normal path; bounded on the abort path).
       volatile int no_abort = 0;
-      mbar_wait(bar_q, 0, &no_abort, p.status);
-      for (int j = max(0, issued - kStages); j < issued; ++j) {
-        mbar_wait(bar_k_full(j % kStages), (j / kStages) & 1, &no_abort, p.status);
-        mbar_wait(bar_v_full(j % kStages), (j / kStages) & 1, &no_abort, p.status);
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+      mbar_wait(bar(kBarQ), 0, &no_abort, p.status);
+      for (int j = max(0, issued_k - kStages); j < issued_k; ++j)
+        mbar_wait(bar(kBarKFull + j % kStages), (j / kStages) & 1, &no_abort, p.status);
+      for (int j = max(0, issued_v - kStages); j < issued_v; ++j)
+        mbar_wait(bar(kBarVFull + j % kStages), (j / kStages) & 1, &no_abort, p.status);
+    } else if (warp == 1 && lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
       constexpr uint32_t idesc_s = idesc_bf16_f32(kBlockM, kBlockN, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(kBlockM, D, false, true);
-      bool ok = mbar_wait(bar_q, 0, abort_flag, p.status);
-      auto issue_s = [&](int j) -> bool {
-        const int st = j % kStages, sb = j & 1;
-        if (!mbar_wait(bar_k_full(st), (j / kStages) & 1, abort_flag, p.status)) return false;
-        if (j >= 2 && !mbar_wait(bar_s_free(sb), ((j >> 1) - 1) & 1, abort_flag, p.status)) return false;
-        tc_fence_after();
+      auto issue_s = [&](int x, int st) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kPanelBytes + (kk & 3) * 32;
-          const uint64_t a = smem_desc_sw128(sQ + off, 16, 1024);
+          const uint64_t a = smem_desc_sw128(sQ + x * kTileBytes + off, 16, 1024);
           const uint64_t b = smem_desc_sw128(sK + st * kTileBytes + off, 16, 1024);
-          mma_bf16_ss(tmem_S0 + sb * kBlockN, a, b, idesc_s, kk > 0 ? 1u : 0u);
+          mma_bf16_ss(tmem + x * kBlockN, a, b, idesc_s, kk > 0 ? 1u : 0u);
         }
-        mma_commit(bar_s_full(sb));
-        return true;
       };
-      if (ok && n > 0) ok = issue_s(0);
-      for (int j = 0; ok && j < n; ++j) {
-        if (j + 1 < n && !(ok = issue_s(j + 1))) break;
-        const int st = j % kStages;
-        if (!(ok = mbar_wait(bar_p_full, j & 1, abort_flag, p.status))) break;
-        if (!(ok = mbar_wait(bar_v_full(st), (j / kStages) & 1, abort_flag, p.status))) break;
-        tc_fence_after();
+      auto issue_pv = [&](int x, int st, bool first) {
 #pragma unroll
         for (int kk = 0; kk < kBlockN / 16; ++kk) {
-          const uint64_t a = smem_desc_sw128(sP + (kk >> 2) * kPanelBytes + (kk & 3) * 32, 16, 1024);
           const uint64_t b = smem_desc_sw128(sV + st * kTileBytes + kk * 2048, kPanelBytes, 1024);
-          mma_bf16_ss(tmem_O, a, b, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(tmem + 256 + x * D, tmem + x * kBlockN + kk * 8, b, idesc_o, (!first || kk > 0) ? 1u : 0u);
         }
-        mma_commit(bar_o_done);
-        if (j + kStages < n) mma_commit(bar_kv_empty(st));
+      };
+      bool ok = mbar_wait(bar(kBarQ), 0, abort_flag, p.status);
+      for (int j = 0; ok && j < n; ++j) {
+        const int st = j % kStages, pst = (j + kStages - 1) % kStages;
+        if (!(ok = mbar_wait(bar(kBarKFull + st), (j / kStages) & 1, abort_flag, p.status))) break;
+        if (j > 0 && !(ok = mbar_wait(bar(kBarVFull + pst), ((j - 1) / kStages) & 1, abort_flag, p.status))) break;
+        for (int x = 0; x < n_act; ++x) {
+          if (j > 0) {
+            if (!(ok = mbar_wait(bar(kBarPFull + x), (j - 1) & 1, abort_flag, p.status))) break;
+            tc_fence_after();
+            issue_pv(x, pst, j == 1);
+          } else {
+            tc_fence_after();
+          }
+          issue_s(x, st);
+          mma_commit(bar(kBarSFull + x));
+        }
+        if (!ok) break;
+        if (j + kStages < n) mma_commit(bar(kBarKEmpty + st));
+        if (j > 0 && (j - 1) + kStages < n) mma_commit(bar(kBarVEmpty + pst));
+      }
+      if (ok && n > 0) {
+        const int pst = (n - 1) % kStages;
+        ok = mbar_wait(bar(kBarVFull + pst), ((n - 1) / kStages) & 1, abort_flag, p.status);
+        for (int x = 0; ok && x < n_act; ++x) {
+          if (!(ok = mbar_wait(bar(kBarPFull + x), (n - 1) & 1, abort_flag, p.status))) break;
+          tc_fence_after();
+          issue_pv(x, pst, n == 1);
+          mma_commit(bar(kBarODone + x));
+        }
       }
       // Drain: all MMAs of this thread complete before TMEM is released.
-      mma_commit(bar_drain);
+      mma_commit(bar(kBarDrain));
       volatile int no_abort = 0;
-      mbar_wait(bar_drain, 0, &no_abort, p.status);
+      mbar_wait(bar(kBarDrain), 0, &no_abort, p.status);
     }
-  } else if (warp >= 4) {
+  } else {
+    setmaxnreg_inc224();
     // ------------------------------------------------------------ softmax
-    const int r = threadIdx.x - 128;                 // query row = TMEM lane
+    const int x = (warp >> 2) - 1;                    // query tile 0 (A) or 1 (B)
+    const int r = threadIdx.x - 128 * (x + 1);        // row within the tile = TMEM lane
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + x * kBlockN + lane_base;
+    const uint32_t tO = tmem + 256 + x * D + lane_base;
+    const bool active = x < n_act;
     const float qk2 = p.tau[it.h] * p.scale_log2;
     const float* bias_h = p.bias ? p.bias + it.h * p.sc.S : nullptr;
+    float* mrow = mass_sm + (x * p.sc.S) * kBlockM + r;   // [s] stride kBlockM
     float m_used = -INFINITY, l_sum = 0.f;
     if (MASS)
-      for (int s = 0; s < p.sc.S; ++s) mass_sm[s * kBlockM + r] = 0.f;
-    bool ok = true;
-    const uint32_t prow = uint32_t(r) * 128u;
-    const uint32_t rsw = uint32_t(r & 7);
+      for (int s = 0; s < p.sc.S; ++s) mrow[s * kBlockM] = 0.f;
+    bool ok = active;
 
-    for (int j = 0; j < n; ++j) {
-      const int sb = j & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full(sb), (j >> 1) & 1, abort_flag, p.status));
+    for (int j = 0; ok && j < n; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarSFull + x), j & 1, abort_flag, p.status));
       if (!ok) break;
       tc_fence_after();
-      float x[kBlockN];
+      float sv[kBlockN];
       {
         uint32_t v[kBlockN / 32][32];
 #pragma unroll
-        for (int c = 0; c < kBlockN / 32; ++c) tmem_ld32(tmem_S0 + sb * kBlockN + c * 32 + lane_base, v[c]);
+        for (int c = 0; c < kBlockN / 32; ++c) tmem_ld32(tS + c * 32, v[c]);
         tmem_wait_ld();
 #pragma unroll
         for (int c = 0; c < kBlockN / 32; ++c) {
           reg_fence32(v[c]);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) x[c * 32 + i] = __uint_as_float(v[c][i]);
+          for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(v[c][i]);
         }
       }
-      tc_fence_before();
-      mbar_arrive(bar_s_free(sb));
-
       const KTile t = it.tile(p, j);
-      // logits in the log2 domain, bias per source-scale segment, mask tail
       int nseg = 0, seg_scale = 0;
       for_each_segment<PRUNED>(p, it, t, [&](int, int, int s) { ++nseg; seg_scale = s; });
-      if (nseg == 1) {
+      const bool fast = (nseg == 1) && (t.valid == kBlockN) && (qk2 > 0.f);
+      float m_tile;
+      float shift;  // exponent argument = sv * qk2 + shift (fast) or sv - m_used (general)
+      if (fast) {
+        float m0 = sv[0], m1 = sv[1], m2 = sv[2], m3 = sv[3];
+#pragma unroll
+        for (int c = 4; c < kBlockN; c += 8) {
+          m0 = fmax3(m0, sv[c + 0], sv[c + 1]);
+          m1 = fmax3(m1, sv[c + 2], sv[c + 3]);
+          m2 = fmax3(m2, sv[c + 4], sv[c + 5]);
+          if (c + 7 < kBlockN) m3 = fmax3(m3, sv[c + 6], sv[c + 7]);
+          else m3 = fmaxf(m3, sv[c + 6]);
+        }
         const float b2 = bias_h ? bias_h[seg_scale] * kLog2e : 0.f;
-#pragma unroll
-        for (int c = 0; c < kBlockN; ++c) x[c] = (c < t.valid) ? fmaf(x[c], qk2, b2) : -INFINITY;
+        m_tile = fmaf(fmaxf(fmax3(m0, m1, m2), m3), qk2, b2);
+        shift = b2;
       } else {
+        // logits in the log2 domain with per-segment bias, tail masked
 #pragma unroll
-        for (int c = 0; c < kBlockN; ++c) x[c] = (c < t.valid) ? x[c] * qk2 : -INFINITY;
+        for (int c = 0; c < kBlockN; ++c) sv[c] = (c < t.valid) ? sv[c] * qk2 : -INFINITY;
         if (bias_h) {
           for_each_segment<PRUNED>(p, it, t, [&](int cb, int ce, int s) {
             const float b2 = bias_h[s] * kLog2e;
 #pragma unroll
-            for (int c = 0; c < kBlockN; ++c) x[c] += (c >= cb && c < ce) ? b2 : 0.f;
+            for (int c = 0; c < kBlockN; ++c) sv[c] += (c >= cb && c < ce) ? b2 : 0.f;
           });
         }
-      }
-      float m_tile = x[0];
+        float m0 = sv[0], m1 = sv[1], m2 = sv[2], m3 = sv[3];
 #pragma unroll
-      for (int c = 1; c < kBlockN; ++c) m_tile = fmaxf(m_tile, x[c]);
-
-      // PV_{j-1} complete: the P buffer is free and O is stable.
-      if (j > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar_o_done, (j - 1) & 1, abort_flag, p.status));
-        if (!ok) break;
+        for (int c = 4; c < kBlockN; c += 8) {
+          m0 = fmax3(m0, sv[c + 0], sv[c + 1]);
+          m1 = fmax3(m1, sv[c + 2], sv[c + 3]);
+          m2 = fmax3(m2, sv[c + 4], sv[c + 5]);
+          if (c + 7 < kBlockN) m3 = fmax3(m3, sv[c + 6], sv[c + 7]);
+          else m3 = fmaxf(m3, sv[c + 6]);
+        }
+        m_tile = fmaxf(fmax3(m0, m1, m2), m3);
+        shift = 0.f;
       }
-      // Rescale when this row's max grew past the threshold; the TMEM access
-      // is warp-collective, so a warp rescales if any of its rows must.
-      bool rescaled = false;
+      // Running max with a stale-max threshold; O_X is stable here (the
+      // commit that completed S_X(j) also covers PV_X(j-1)).
       float f = 1.f;
       if (j == 0) {
         m_used = m_tile;
@@ -383,70 +427,82 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         m_used = m_tile;
         l_sum *= f;
         if (MASS)
-          for (int s = 0; s <= it.k; ++s) mass_sm[s * kBlockM + r] *= f;
+          for (int s = 0; s <= it.k; ++s) mrow[s * kBlockM] *= f;
       }
       if (j > 0 && __any_sync(0xffffffffu, f != 1.f)) {
-        tc_fence_after();
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t v[32];
-          tmem_ld32(tmem_O + c * 32 + lane_base, v);
+          tmem_ld32(tO + c * 32, v);
           tmem_wait_ld();
           reg_fence32(v);
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
-          tmem_st32(tmem_O + c * 32 + lane_base, v);
+          tmem_st32(tO + c * 32, v);
         }
-        rescaled = true;
       }
-      float tile_sum = 0.f;
+      // p = 2^(argument - m_used)
+      if (fast) {
+        const float sh = shift - m_used;
 #pragma unroll
-      for (int c = 0; c < kBlockN; ++c) {
-        x[c] = ex2_approx(x[c] - m_used);
-        tile_sum += x[c];
+        for (int c = 0; c < kBlockN; c += 2) ffma2(sv[c], sv[c + 1], sv[c], sv[c + 1], qk2, qk2, sh, sh);
+      } else {
+        const float sh = -m_used;
+#pragma unroll
+        for (int c = 0; c < kBlockN; c += 2) fadd2(sv[c], sv[c + 1], sv[c], sv[c + 1], sh, sh);
       }
+#pragma unroll
+      for (int c = 0; c < kBlockN; ++c) sv[c] = ex2_approx(sv[c]);
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f, a4 = 0.f, a5 = 0.f, a6 = 0.f, a7 = 0.f;
+#pragma unroll
+      for (int c = 0; c < kBlockN; c += 8) {
+        fadd2(a0, a1, a0, a1, sv[c + 0], sv[c + 1]);
+        fadd2(a2, a3, a2, a3, sv[c + 2], sv[c + 3]);
+        fadd2(a4, a5, a4, a5, sv[c + 4], sv[c + 5]);
+        fadd2(a6, a7, a6, a7, sv[c + 6], sv[c + 7]);
+      }
+      const float tile_sum = ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
       l_sum += tile_sum;
       if (MASS) {
         if (nseg == 1) {
-          mass_sm[seg_scale * kBlockM + r] += tile_sum;
+          mrow[seg_scale * kBlockM] += tile_sum;
         } else {
           for_each_segment<PRUNED>(p, it, t, [&](int cb, int ce, int s) {
             float acc = 0.f;
 #pragma unroll
-            for (int c = 0; c < kBlockN; ++c) acc += (c >= cb && c < ce) ? x[c] : 0.f;
-            mass_sm[s * kBlockM + r] += acc;
+            for (int c = 0; c < kBlockN; ++c) acc += (c >= cb && c < ce) ? sv[c] : 0.f;
+            mrow[s * kBlockM] += acc;
           });
         }
       }
-      // P row -> shared memory, 128-byte swizzled K-major operand layout
+      // P_X (bf16 pairs) over the first 64 columns of S_X
+      {
+        uint32_t pk[2][32];
 #pragma unroll
-      for (int q = 0; q < kBlockN / 8; ++q) {
-        const uint32_t addr = sP + (q >> 3) * kPanelBytes + prow + ((uint32_t(q & 7) ^ rsw) << 4);
-        const uint32_t w0 = pack_bf16x2(x[8 * q + 0], x[8 * q + 1]);
-        const uint32_t w1 = pack_bf16x2(x[8 * q + 2], x[8 * q + 3]);
-        const uint32_t w2 = pack_bf16x2(x[8 * q + 4], x[8 * q + 5]);
-        const uint32_t w3 = pack_bf16x2(x[8 * q + 6], x[8 * q + 7]);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w0), "r"(w1), "r"(w2), "r"(w3)
-                     : "memory");
+        for (int c = 0; c < 32; ++c) {
+          pk[0][c] = pack_bf16x2(sv[2 * c], sv[2 * c + 1]);
+          pk[1][c] = pack_bf16x2(sv[64 + 2 * c], sv[64 + 2 * c + 1]);
+        }
+        tmem_st32(tS, pk[0]);
+        tmem_st32(tS + 32, pk[1]);
       }
-      fence_proxy_async_smem();
-      if (rescaled) tmem_wait_st();
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar_p_full);
+      mbar_arrive(bar(kBarPFull + x));
     }
 
     // ---------------------------------------------------------- epilogue
-    if (ok && n > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar_o_done, (n - 1) & 1, abort_flag, p.status));
-    const bool row_ok = ok && r < it.rows_valid;
+    if (ok && n > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarODone + x), 0, abort_flag, p.status));
+    const bool row_ok = ok && r < it.rows_valid[x];
     const float inv_l = 1.f / l_sum;
     if (ok && p.out != nullptr) {
       tc_fence_after();
-      const int out_row = (p.q_scale_rows ? 0 : p.sc.off[it.k]) + it.qrow0 + r;
+      const int out_row = (p.q_scale_rows ? 0 : p.sc.off[it.k]) + it.row0 + x * kBlockM + r;
       uint16_t* orow = p.out + (int64_t(it.bh) * p.q_rows + out_row) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t v[32];
-        tmem_ld32(tmem_O + c * 32 + lane_base, v);
+        tmem_ld32(tO + c * 32, v);
         tmem_wait_ld();
         reg_fence32(v);
         if (row_ok) {
@@ -463,17 +519,20 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       }
     }
     if (MASS) {
-      // mean over the B * n_k rows of scale k of m_i(s), one atomic per (h, s, k)
-      const float inv_rows = 1.f / (float(p.B) * float(p.sc.n[it.k]));
+      // mean over the B * n_k rows of scale k of m_i(s): both tiles' rows are
+      // reduced in the CTA, then one atomic per (h, s, k)
       for (int s = 0; s <= it.k; ++s) {
-        float v = row_ok ? mass_sm[s * kBlockM + r] * inv_l : 0.f;
+        float v = row_ok ? mrow[s * kBlockM] * inv_l : 0.f;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) red_sm[(warp & 3) * 32 + s] = v;
+        if (lane == 0) red_sm[(x * 4 + (warp & 3)) * 32 + s] = v;
       }
-      named_bar_sync(1, kBlockM);
-      if (ok && r <= it.k) {
-        const float tot = red_sm[r] + red_sm[32 + r] + red_sm[64 + r] + red_sm[96 + r];
+      named_bar_sync(1, 2 * kBlockM);
+      if (x == 0 && r <= it.k && *abort_flag == 0) {
+        float tot = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) tot += red_sm[w * 32 + r];
+        const float inv_rows = 1.f / (float(p.B) * float(p.sc.n[it.k]));
         atomicAdd(p.mass + (int64_t(it.h) * p.sc.S + r) * p.sc.S + it.k, tot * inv_rows);
       }
     }
@@ -500,18 +559,20 @@ static int encode_rows(CUtensorMap* m, const uint16_t* base, int D, int64_t rows
   return encode_bf16_map(m, base, 2, dims, strides, 128);
 }
 
-// Query-tile kinds of the selected scales, heaviest (most keys) first.
+// Query-tile pairs (256 rows of one scale) of the selected scales, heaviest
+// (most keys) first within each (batch, head).
 static int build_qtiles(Params& p, int query_scale) {
   struct E { int64_t w; uint32_t v; };
   std::vector<E> e;
   for (int k = 0; k < p.sc.S; ++k) {
     if (query_scale >= 0 && k != query_scale) continue;
-    for (int r = 0; r < p.sc.n[k]; r += kBlockM) e.push_back({int64_t(p.sc.off[k]) + p.sc.n[k], (uint32_t(k) << 24) | uint32_t(r)});
+    for (int r = 0; r < p.sc.n[k]; r += 2 * kBlockM)
+      e.push_back({int64_t(p.sc.off[k]) + p.sc.n[k], (uint32_t(k) << 24) | uint32_t(r)});
   }
-  if (e.empty() || int(e.size()) > kMaxQTiles) return VARK_E_SHAPE;
+  if (e.empty() || int(e.size()) > kMaxPairs) return VARK_E_SHAPE;
   std::stable_sort(e.begin(), e.end(), [](const E& a, const E& b) { return a.w > b.w; });
-  p.n_qt = int(e.size());
-  for (int i = 0; i < p.n_qt; ++i) p.qt[i] = e[i].v;
+  p.n_pairs = int(e.size());
+  for (int i = 0; i < p.n_pairs; ++i) p.pair[i] = e[i].v;
   return VARK_OK;
 }
 
@@ -519,12 +580,12 @@ template <int D, bool PRUNED, bool MASS>
 static int launch(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& kc,
                   const CUtensorMap& vc, const Params& p, cudaStream_t st) {
   auto kern = attn_kernel<D, PRUNED, MASS>;
-  const int smem = Smem<D>::kAlloc;
+  const int smem = Smem<D>::alloc(MASS, p.sc.S);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
     cudaGetLastError();
     return VARK_E_CUDA;
   }
-  const int64_t grid = int64_t(p.n_qt) * p.B * p.H;
+  const int64_t grid = int64_t(p.n_pairs) * p.B * p.H;
   if (grid > INT32_MAX) return VARK_E_SHAPE;
   kern<<<unsigned(grid), kThreads, smem, st>>>(q, k, v, kc, vc, p);
   return cudaGetLastError() == cudaSuccess ? VARK_OK : VARK_E_CUDA;
