@@ -47,9 +47,16 @@ constexpr int kBlockN = 128;
 constexpr int kStages = 2;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxPairs = 512;
+constexpr int kMaxDesc = 256;            // key tiles with a precomputed descriptor
 constexpr int kPanelBytes = 128 * 128;   // 128 rows x 128 bytes (64 bf16)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 domain
+// Of every 8 columns of a full single-segment tile, this many take 2^x from the
+// FMA-pipe polynomial and the rest from MUFU ex2.  MUFU alone matches the
+// tensor pipe's time per score at D = 128, but measured on B200 the softmax
+// is bound by instruction issue, not MUFU: shares of 2, 4, 6 per 8 ran 5-17%
+// slower than 0, so the polynomial path is off.
+constexpr int kPolyPer8 = 0;
 
 struct Params {
   ScaleTable sc;
@@ -94,7 +101,11 @@ struct Smem {
   static constexpr int kBar = kV + kStages * kTile;
   static constexpr int kMisc = kBar + kNumBars * 8;     // tmem base, abort flag
   static constexpr int kRed = kMisc + 16;               // [2 tiles][4 warps][32] fp32
-  static constexpr int kMass = kRed + 2 * 4 * 32 * 4;   // [2 tiles][S][128] fp32 (calibration)
+  static constexpr int kDesc = kRed + 2 * 4 * 32 * 4;   // [kMaxDesc] uint32 key-tile descriptors
+  static constexpr int kBias2 = kDesc + kMaxDesc * 4;   // [32] fp32 bias * log2(e) of this head
+  static constexpr int kSegOff = kBias2 + 32 * 4;       // [32] int32 this head's seg_off (pruned)
+  static constexpr int kColBias = kSegOff + 32 * 4;     // [2 tiles][128] fp32 per-column bias / mask
+  static constexpr int kMass = kColBias + 2 * 128 * 4;  // [2 tiles][S][128] fp32 (calibration)
   static int alloc(bool mass, int S) { return kMass + (mass ? 2 * S * kBlockM * 4 : 0) + 1024; }
 };
 
@@ -169,9 +180,11 @@ __device__ Item<PRUNED> decode_item(const Params& p) {
 }
 
 // Calls f(col_begin, col_end, scale) for every source-scale segment of the
-// valid columns of a key tile, in column order.
+// valid columns of a key tile, in column order.  segoff: this head's seg_off
+// row (pruned attention).
 template <bool PRUNED, typename F>
-__device__ __forceinline__ void for_each_segment(const Params& p, const Item<PRUNED>& it, const KTile& t, F&& f) {
+__device__ __forceinline__ void for_each_segment(const Params& p, const Item<PRUNED>& it, const KTile& t,
+                                                 const int32_t* segoff, F&& f) {
   if (!PRUNED) {
     const int lo = t.key0, hi = t.key0 + t.valid;
     for (int s = 0; s <= it.k; ++s) {
@@ -181,7 +194,7 @@ __device__ __forceinline__ void for_each_segment(const Params& p, const Item<PRU
   } else if (t.src == 1) {
     const int lo = t.key0, hi = t.key0 + t.valid;
     for (int s = 0; s < it.k; ++s) {
-      const int so = p.seg_off[it.h * p.sc.S + s];
+      const int so = segoff[s];
       if (so < 0) continue;
       const int a = max(so, lo), e = min(so + p.sc.n[s], hi);
       if (a < e) f(a - lo, e - lo, s);
@@ -189,6 +202,37 @@ __device__ __forceinline__ void for_each_segment(const Params& p, const Item<PRU
   } else {
     f(0, t.valid, it.k);
   }
+}
+
+// Key-tile descriptor: bit 0 = one source scale and all 128 columns valid;
+// bits 8..15 = that scale; bits 16..31 = valid columns.
+template <bool PRUNED>
+__device__ __forceinline__ uint32_t make_desc(const Params& p, const Item<PRUNED>& it, int j,
+                                              const int32_t* segoff) {
+  const KTile t = it.tile(p, j);
+  int nseg = 0, sc = 0;
+  for_each_segment<PRUNED>(p, it, t, segoff, [&](int, int, int s) { ++nseg; sc = s; });
+  return uint32_t(nseg == 1 && t.valid == kBlockN) | (uint32_t(sc) << 8) | (uint32_t(t.valid) << 16);
+}
+
+// Source scale of column c of a key tile (c < valid).
+template <bool PRUNED>
+__device__ __forceinline__ int column_scale(const Params& p, const Item<PRUNED>& it, const KTile& t, int c,
+                                            const int32_t* segoff) {
+  const int key = t.key0 + c;
+  if (!PRUNED) {
+    int s = 0;
+    while (s < it.k && key >= p.sc.off[s + 1]) ++s;
+    return s;
+  } else if (t.src == 1) {
+    int sc = 0;
+    for (int s = 0; s < it.k; ++s) {
+      const int so = segoff[s];
+      if (so >= 0 && key >= so && key < so + p.sc.n[s]) sc = s;
+    }
+    return sc;
+  }
+  return it.k;
 }
 
 template <int D, bool PRUNED, bool MASS>
@@ -346,20 +390,40 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     // ------------------------------------------------------------ softmax
     const int x = (warp >> 2) - 1;                    // query tile 0 (A) or 1 (B)
     const int r = threadIdx.x - 128 * (x + 1);        // row within the tile = TMEM lane
+    const int t256 = threadIdx.x - 128;
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + x * kBlockN + lane_base;
     const uint32_t tO = tmem + 256 + x * D + lane_base;
     const bool active = x < n_act;
     const float qk2 = p.tau[it.h] * p.scale_log2;
-    const float* bias_h = p.bias ? p.bias + it.h * p.sc.S : nullptr;
+    uint32_t* desc_sm = reinterpret_cast<uint32_t*>(smem + L::kDesc);
+    float* bias2_sm = reinterpret_cast<float*>(smem + L::kBias2);
+    int32_t* segoff_sm = reinterpret_cast<int32_t*>(smem + L::kSegOff);
+    float* colbias = reinterpret_cast<float*>(smem + L::kColBias) + x * kBlockN;
     float* mrow = mass_sm + (x * p.sc.S) * kBlockM + r;   // [s] stride kBlockM
+
+    // Per-CTA tables, shared by both tiles: bias * log2(e) per source scale,
+    // this head's seg_off row, and the descriptor of every key tile.
+    if (t256 < p.sc.S) {
+      bias2_sm[t256] = p.bias ? p.bias[it.h * p.sc.S + t256] * kLog2e : 0.f;
+      if (PRUNED) segoff_sm[t256] = p.seg_off[it.h * p.sc.S + t256];
+    }
+    named_bar_sync(2, 2 * kBlockM);
+    for (int jj = t256; jj < min(n, kMaxDesc); jj += 2 * kBlockM) desc_sm[jj] = make_desc<PRUNED>(p, it, jj, segoff_sm);
+    named_bar_sync(2, 2 * kBlockM);
+
     float m_used = -INFINITY, l_sum = 0.f;
     if (MASS)
       for (int s = 0; s < p.sc.S; ++s) mrow[s * kBlockM] = 0.f;
     bool ok = active;
 
     for (int j = 0; ok && j < n; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarSFull + x), j & 1, abort_flag, p.status));
+      const uint32_t d = j < kMaxDesc ? desc_sm[j] : make_desc<PRUNED>(p, it, j, segoff_sm);
+      const bool fast = (d & 1u) && (qk2 > 0.f);
+      const int seg_scale = int((d >> 8) & 0xFFu);
+      // the tile's 128 threads agree on continuing (a per-column table and a
+      // named barrier may follow)
+      ok = bar_and(3 + x, kBlockM, mbar_wait(bar(kBarSFull + x), j & 1, abort_flag, p.status));
       if (!ok) break;
       tc_fence_after();
       float sv[kBlockN];
@@ -375,47 +439,46 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(v[c][i]);
         }
       }
-      const KTile t = it.tile(p, j);
-      int nseg = 0, seg_scale = 0;
-      for_each_segment<PRUNED>(p, it, t, [&](int, int, int s) { ++nseg; seg_scale = s; });
-      const bool fast = (nseg == 1) && (t.valid == kBlockN) && (qk2 > 0.f);
-      float m_tile;
-      float shift;  // exponent argument = sv * qk2 + shift (fast) or sv - m_used (general)
+      float m_tile, sh;
       if (fast) {
+        // one source scale, all columns valid: exponent = sv * qk2 + (b2 - m)
         float m0 = sv[0], m1 = sv[1], m2 = sv[2], m3 = sv[3];
 #pragma unroll
-        for (int c = 4; c < kBlockN; c += 8) {
+        for (int c = 4; c < kBlockN - 4; c += 8) {
           m0 = fmax3(m0, sv[c + 0], sv[c + 1]);
           m1 = fmax3(m1, sv[c + 2], sv[c + 3]);
           m2 = fmax3(m2, sv[c + 4], sv[c + 5]);
-          if (c + 7 < kBlockN) m3 = fmax3(m3, sv[c + 6], sv[c + 7]);
-          else m3 = fmaxf(m3, sv[c + 6]);
+          m3 = fmax3(m3, sv[c + 6], sv[c + 7]);
         }
-        const float b2 = bias_h ? bias_h[seg_scale] * kLog2e : 0.f;
-        m_tile = fmaf(fmaxf(fmax3(m0, m1, m2), m3), qk2, b2);
-        shift = b2;
+        m0 = fmax3(m0, sv[kBlockN - 4], sv[kBlockN - 3]);
+        m1 = fmax3(m1, sv[kBlockN - 2], sv[kBlockN - 1]);
+        const float b2 = bias2_sm[seg_scale];
+        m_tile = fmaf(fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)), qk2, b2);
+        sh = b2;
       } else {
-        // logits in the log2 domain with per-segment bias, tail masked
+        // boundary / tail tile: per-column bias (or -inf mask) from a table
+        // the tile's 128 threads fill, one column each
+        const KTile t = it.tile(p, j);
+        colbias[r] = (r < t.valid) ? bias2_sm[column_scale<PRUNED>(p, it, t, r, segoff_sm)] : -INFINITY;
+        named_bar_sync(3 + x, kBlockM);
 #pragma unroll
-        for (int c = 0; c < kBlockN; ++c) sv[c] = (c < t.valid) ? sv[c] * qk2 : -INFINITY;
-        if (bias_h) {
-          for_each_segment<PRUNED>(p, it, t, [&](int cb, int ce, int s) {
-            const float b2 = bias_h[s] * kLog2e;
-#pragma unroll
-            for (int c = 0; c < kBlockN; ++c) sv[c] += (c >= cb && c < ce) ? b2 : 0.f;
-          });
+        for (int c = 0; c < kBlockN; c += 4) {
+          const float4 cb = *reinterpret_cast<const float4*>(colbias + c);
+          ffma2(sv[c], sv[c + 1], sv[c], sv[c + 1], qk2, qk2, cb.x, cb.y);
+          ffma2(sv[c + 2], sv[c + 3], sv[c + 2], sv[c + 3], qk2, qk2, cb.z, cb.w);
         }
         float m0 = sv[0], m1 = sv[1], m2 = sv[2], m3 = sv[3];
 #pragma unroll
-        for (int c = 4; c < kBlockN; c += 8) {
+        for (int c = 4; c < kBlockN - 4; c += 8) {
           m0 = fmax3(m0, sv[c + 0], sv[c + 1]);
           m1 = fmax3(m1, sv[c + 2], sv[c + 3]);
           m2 = fmax3(m2, sv[c + 4], sv[c + 5]);
-          if (c + 7 < kBlockN) m3 = fmax3(m3, sv[c + 6], sv[c + 7]);
-          else m3 = fmaxf(m3, sv[c + 6]);
+          m3 = fmax3(m3, sv[c + 6], sv[c + 7]);
         }
-        m_tile = fmaxf(fmax3(m0, m1, m2), m3);
-        shift = 0.f;
+        m0 = fmax3(m0, sv[kBlockN - 4], sv[kBlockN - 3]);
+        m1 = fmax3(m1, sv[kBlockN - 2], sv[kBlockN - 1]);
+        m_tile = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+        sh = 0.f;
       }
       // Running max with a stale-max threshold; O_X is stable here (the
       // commit that completed S_X(j) also covers PV_X(j-1)).
@@ -441,18 +504,25 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           tmem_st32(tO + c * 32, v);
         }
       }
-      // p = 2^(argument - m_used)
+      // p = 2^(exponent - m_used)
       if (fast) {
-        const float sh = shift - m_used;
+        const float shm = sh - m_used;
 #pragma unroll
-        for (int c = 0; c < kBlockN; c += 2) ffma2(sv[c], sv[c + 1], sv[c], sv[c + 1], qk2, qk2, sh, sh);
+        for (int c = 0; c < kBlockN; c += 2) ffma2(sv[c], sv[c + 1], sv[c], sv[c + 1], qk2, qk2, shm, shm);
+#pragma unroll
+        for (int c = 0; c < kBlockN; c += 8) {
+#pragma unroll
+          for (int i = 0; i < kPolyPer8; i += 2) exp2_poly2(sv[c + i], sv[c + i + 1]);
+#pragma unroll
+          for (int i = kPolyPer8; i < 8; ++i) sv[c + i] = ex2_approx(sv[c + i]);
+        }
       } else {
-        const float sh = -m_used;
+        const float shm = -m_used;
 #pragma unroll
-        for (int c = 0; c < kBlockN; c += 2) fadd2(sv[c], sv[c + 1], sv[c], sv[c + 1], sh, sh);
+        for (int c = 0; c < kBlockN; c += 2) fadd2(sv[c], sv[c + 1], sv[c], sv[c + 1], shm, shm);
+#pragma unroll
+        for (int c = 0; c < kBlockN; ++c) sv[c] = ex2_approx(sv[c]);
       }
-#pragma unroll
-      for (int c = 0; c < kBlockN; ++c) sv[c] = ex2_approx(sv[c]);
       float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f, a4 = 0.f, a5 = 0.f, a6 = 0.f, a7 = 0.f;
 #pragma unroll
       for (int c = 0; c < kBlockN; c += 8) {
@@ -464,14 +534,18 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       const float tile_sum = ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
       l_sum += tile_sum;
       if (MASS) {
-        if (nseg == 1) {
+        if (d & 1u) {
           mrow[seg_scale * kBlockM] += tile_sum;
         } else {
-          for_each_segment<PRUNED>(p, it, t, [&](int cb, int ce, int s) {
-            float acc = 0.f;
+          const KTile t = it.tile(p, j);
+          for_each_segment<PRUNED>(p, it, t, segoff_sm, [&](int cb, int ce, int s) {
+            float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-            for (int c = 0; c < kBlockN; ++c) acc += (c >= cb && c < ce) ? sv[c] : 0.f;
-            mrow[s * kBlockM] += acc;
+            for (int c = 0; c < kBlockN; c += 2) {
+              acc0 += (unsigned(c - cb) < unsigned(ce - cb)) ? sv[c] : 0.f;
+              acc1 += (unsigned(c + 1 - cb) < unsigned(ce - cb)) ? sv[c + 1] : 0.f;
+            }
+            mrow[s * kBlockM] += acc0 + acc1;
           });
         }
       }

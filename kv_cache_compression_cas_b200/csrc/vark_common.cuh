@@ -93,32 +93,61 @@ VARK_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait that may suspend the thread until the phase completes (or the
+// hinted time passes), so waiting warps do not take issue slots from the
+// warps that work.
+constexpr uint32_t kSuspendHintNs = 10000;
+VARK_DEV bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase with the given parity to complete.  Gives up after
 // kWaitLimitNs: sets *abort_flag (shared) and the caller's status word, and
-// returns false.  Also returns false at once when another role has aborted.
+// returns false.  Also returns false at once when another role has aborted
+// or another CTA of the launch has recorded an error.
 VARK_DEV bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int32_t* status) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (*abort_flag) return false;
-      // Another CTA of the launch already gave up: stop too.
-      if (status && *reinterpret_cast<volatile int32_t*>(status) != 0) {
-        *abort_flag = 1;
-        return false;
-      }
-      if (globaltimer() - t0 > kWaitLimitNs) {
-        *abort_flag = 1;
-        if (status) atomicExch(status, VARK_E_TIMEOUT);
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_wait_suspend(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (status && *reinterpret_cast<volatile int32_t*>(status) != 0) {
+      *abort_flag = 1;
+      return false;
+    }
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      if (status) atomicExch(status, VARK_E_TIMEOUT);
+      return false;
     }
   }
 }
 
 VARK_DEV void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Named barrier that also ANDs a predicate over the participating threads:
+// every thread gets the same answer, so a group can agree to stop together.
+VARK_DEV bool bar_and(int id, int count, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %3, 0;\n\t"
+      "bar.red.and.pred p, %1, %2, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(id), "r"(count), "r"(uint32_t(v))
+      : "memory");
+  return r != 0;
 }
 
 VARK_DEV void named_bar_sync(int id, int count) {
@@ -272,6 +301,28 @@ VARK_DEV void fadd2(float& d0, float& d1, float a0, float a1, float b0, float b1
       "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
       : "=f"(d0), "=f"(d1)
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// 2^x for a pair on the FMA pipe.  Range reduction x = n + f with
+// n = round(x) (adding 1.5 * 2^23 leaves n in the low mantissa bits), so
+// f = x - n lies in [-1/2, 1/2]; 2^f comes from the degree-3 minimax
+// polynomial in relative error (max 7.5e-5) fitted by csrc/fit_exp2.py, and
+// 2^n is added into the exponent field.  x is clamped below at -125 (results stay normal fp32 numbers).
+VARK_DEV void exp2_poly2(float& a, float& b) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c0 = 0.9999280571937561f, c1 = 0.6932609677314758f;
+  constexpr float c2 = 0.2426111251115799f, c3 = 0.0551716685295105f;
+  a = fmaxf(a, -125.f);
+  b = fmaxf(b, -125.f);
+  float ta, tb, ra, rb, fa, fb, pa, pb;
+  fadd2(ta, tb, a, b, kMagic, kMagic);
+  fadd2(ra, rb, ta, tb, -kMagic, -kMagic);
+  ffma2(fa, fb, ra, rb, -1.f, -1.f, a, b);
+  ffma2(pa, pb, fa, fb, c3, c3, c2, c2);
+  ffma2(pa, pb, pa, pb, fa, fb, c1, c1);
+  ffma2(pa, pb, pa, pb, fa, fb, c0, c0);
+  a = __uint_as_float(__float_as_uint(pa) + (__float_as_uint(ta) << 23));
+  b = __uint_as_float(__float_as_uint(pb) + (__float_as_uint(tb) << 23));
 }
 
 VARK_DEV float ex2_approx(float x) {
