@@ -205,28 +205,32 @@ __device__ __forceinline__ void for_each_segment(const Params& p, const Item<PRU
 }
 
 // Key-tile descriptor: bit 0 = one source scale and all 128 columns valid;
-// bits 8..15 = that scale; bits 16..31 = valid columns.
+// bits 8..15 = the scale of the first column; bits 16..31 = valid columns.
 template <bool PRUNED>
 __device__ __forceinline__ uint32_t make_desc(const Params& p, const Item<PRUNED>& it, int j,
                                               const int32_t* segoff) {
   const KTile t = it.tile(p, j);
-  int nseg = 0, sc = 0;
-  for_each_segment<PRUNED>(p, it, t, segoff, [&](int, int, int s) { ++nseg; sc = s; });
-  return uint32_t(nseg == 1 && t.valid == kBlockN) | (uint32_t(sc) << 8) | (uint32_t(t.valid) << 16);
+  int nseg = 0, sc = -1;
+  for_each_segment<PRUNED>(p, it, t, segoff, [&](int, int, int s) {
+    ++nseg;
+    if (sc < 0) sc = s;
+  });
+  return uint32_t(nseg == 1 && t.valid == kBlockN) | (uint32_t(max(sc, 0)) << 8) | (uint32_t(t.valid) << 16);
 }
 
-// Source scale of column c of a key tile (c < valid).
+// Source scale of column c of a key tile (c < valid); s0 = the scale of the
+// tile's first column.
 template <bool PRUNED>
 __device__ __forceinline__ int column_scale(const Params& p, const Item<PRUNED>& it, const KTile& t, int c,
-                                            const int32_t* segoff) {
+                                            const int32_t* segoff, int s0) {
   const int key = t.key0 + c;
   if (!PRUNED) {
-    int s = 0;
+    int s = s0;
     while (s < it.k && key >= p.sc.off[s + 1]) ++s;
     return s;
   } else if (t.src == 1) {
-    int sc = 0;
-    for (int s = 0; s < it.k; ++s) {
+    int sc = s0;
+    for (int s = s0; s < it.k; ++s) {
       const int so = segoff[s];
       if (so >= 0 && key >= so && key < so + p.sc.n[s]) sc = s;
     }
@@ -243,8 +247,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
   using L = Smem<D>;
   constexpr int QP = L::kQPanels;
   constexpr uint32_t kTileBytes = L::kTile;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte aligned base, derived from the shared array itself so the
+  // compiler keeps shared-space loads and stores
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(smem);
   const uint32_t sQ = sbase + L::kQ, sK = sbase + L::kK, sV = sbase + L::kV;
   float* red_sm = reinterpret_cast<float*>(smem + L::kRed);
@@ -459,7 +465,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         // boundary / tail tile: per-column bias (or -inf mask) from a table
         // the tile's 128 threads fill, one column each
         const KTile t = it.tile(p, j);
-        colbias[r] = (r < t.valid) ? bias2_sm[column_scale<PRUNED>(p, it, t, r, segoff_sm)] : -INFINITY;
+        colbias[r] = (r < t.valid) ? bias2_sm[column_scale<PRUNED>(p, it, t, r, segoff_sm, seg_scale)] : -INFINITY;
         named_bar_sync(3 + x, kBlockM);
 #pragma unroll
         for (int c = 0; c < kBlockN; c += 4) {
@@ -537,15 +543,22 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         if (d & 1u) {
           mrow[seg_scale * kBlockM] += tile_sum;
         } else {
+          // per source-scale segment: a 0/1 column weight table (one column
+          // per thread) and a dot product with the row's probabilities
           const KTile t = it.tile(p, j);
+          named_bar_sync(3 + x, kBlockM);   // every thread is done with colbias
           for_each_segment<PRUNED>(p, it, t, segoff_sm, [&](int cb, int ce, int s) {
-            float acc0 = 0.f, acc1 = 0.f;
+            colbias[r] = (r >= cb && r < ce) ? 1.f : 0.f;
+            named_bar_sync(3 + x, kBlockM);
+            float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
 #pragma unroll
-            for (int c = 0; c < kBlockN; c += 2) {
-              acc0 += (unsigned(c - cb) < unsigned(ce - cb)) ? sv[c] : 0.f;
-              acc1 += (unsigned(c + 1 - cb) < unsigned(ce - cb)) ? sv[c + 1] : 0.f;
+            for (int c = 0; c < kBlockN; c += 4) {
+              const float4 w4 = *reinterpret_cast<const float4*>(colbias + c);
+              ffma2(acc0, acc1, sv[c], sv[c + 1], w4.x, w4.y, acc0, acc1);
+              ffma2(acc2, acc3, sv[c + 2], sv[c + 3], w4.z, w4.w, acc2, acc3);
             }
-            mrow[s * kBlockM] += acc0 + acc1;
+            mrow[s * kBlockM] += (acc0 + acc1) + (acc2 + acc3);
+            named_bar_sync(3 + x, kBlockM);
           });
         }
       }
