@@ -313,6 +313,18 @@ class CpuSample:
         return flops
 
 
+def reduce_over_ranks(x: float, op: str, world: int, device) -> float:
+    """Max or sum of a host float over all ranks (timing plumbing; no data-path
+    collective).  Works with NCCL (CUDA device) and gloo (CPU device)."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
+    return float(t.item())
+
+
 def profile_case(case: str, reps: int):
     """Small single-kernel runs for Nsight Compute captures (inputs > L2, a
     few GB at most): 'calib' = calibration attention, 4 seeds x 16 heads at
@@ -396,19 +408,8 @@ def main():
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
-    def sum_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.SUM)
-        return float(t.item())
+    max_over_ranks = lambda x: reduce_over_ranks(x, "max", world, dev)
+    sum_over_ranks = lambda x: reduce_over_ranks(x, "sum", world, dev)
 
     w = synth.WORKLOADS[WORKLOAD]
     peaks = _peaks()

@@ -249,6 +249,16 @@ def qkv_key(w: Workload, layer: int, which: str, phase: str) -> int:
     return derive_key(w.base_seed, {"calib": 1, "infer": 2}[phase], layer, {"q": 1, "k": 2, "v": 3}[which])
 
 
+def random_scas(seed: int, layers: int, heads: int, n_scales: int) -> np.ndarray:
+    """Synthetic S-CAS-shaped scores, fp64 [L][H][S], U[0, 1) with the last
+    scale at 0 (no later scale reads it): used where a test needs a schedule at
+    full size without running calibration on the host."""
+    rng = np.random.default_rng([seed, 0x5C])
+    sc = rng.uniform(0.0, 1.0, size=(layers, heads, n_scales))
+    sc[:, :, -1] = 0.0
+    return sc
+
+
 def random_keep(seed: int, heads: int, sides: Sequence[int], budget_bp: int,
                 n_sinks: int, query_scale: int) -> np.ndarray:
     """Seed-random retained-scale sets for the final-scale sweep, uint8
