@@ -26,6 +26,11 @@
  *   - Every call returns a status: VARK_OK (0) or a negative VARK_E_* code.
  *     On an argument error nothing is launched and no output is touched.
  *   - Device pointers and row strides must be 16-byte aligned (VARK_E_ALIGN).
+ *   - Failure-detection test hook (attention calls only; unset in normal use):
+ *     VARK_TEST_WAIT_LIMIT_MS shortens the kernels' bounded waits (default 2 s)
+ *     and VARK_TEST_WITHHOLD_KV_TILE=j makes each CTA's loader stop before key
+ *     tile j, so waits on it run out and the call reports VARK_E_TIMEOUT
+ *     through *dev_status while the CUDA context stays usable.
  *   - Scale lists: `sides[S]` (host) gives the side of each square token map,
  *     ascending; scale s holds n_s = sides[s]^2 tokens, token maps are stored
  *     scale after scale, raster order inside a scale, so

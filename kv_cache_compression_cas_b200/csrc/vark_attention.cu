@@ -34,6 +34,7 @@
 // VARK_E_TIMEOUT in the caller's status word, drains its own async work with
 // bounded waits, frees TMEM and returns.
 #include <algorithm>
+#include <cstdlib>
 #include <vector>
 
 #include "vark_common.cuh"
@@ -76,6 +77,10 @@ struct Params {
   const int32_t* head_off;        // [H]
   const int32_t* seg_off;         // [H][S]
   const int32_t* past_len;        // [H][S]
+  // failure-detection test hook (off by default): wait limit, and a key tile
+  // the producer withholds so that waits on it run out
+  uint64_t wait_limit_ns;
+  int withhold_tile;
 };
 
 enum Bar {
@@ -311,7 +316,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       for (int j = 0; j < n; ++j) {
         const int st = j % kStages;
         const KTile t = it.tile(p, j);
-        if (j >= kStages && !mbar_wait(bar(kBarKEmpty + st), ((j / kStages) - 1) & 1, abort_flag, p.status)) break;
+        if (j == p.withhold_tile) break;   // test hook: this tile never arrives
+        if (j >= kStages && !mbar_wait(bar(kBarKEmpty + st), ((j / kStages) - 1) & 1, abort_flag, p.status, p.wait_limit_ns)) break;
         mbar_arrive_expect_tx(bar(kBarKFull + st), kTileBytes);
         for (int c = 0; c < QP; ++c) {
           const uint32_t dst = sK + st * kTileBytes + c * kPanelBytes;
@@ -319,7 +325,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           else tma_load_2d(dst, &tm_kc, bar(kBarKFull + st), c * 64, t.row);
         }
         issued_k = j + 1;
-        if (j >= kStages && !mbar_wait(bar(kBarVEmpty + st), ((j / kStages) - 1) & 1, abort_flag, p.status)) break;
+        if (j >= kStages && !mbar_wait(bar(kBarVEmpty + st), ((j / kStages) - 1) & 1, abort_flag, p.status, p.wait_limit_ns)) break;
         mbar_arrive_expect_tx(bar(kBarVFull + st), kTileBytes);
         for (int c = 0; c < QP; ++c) {
           const uint32_t dst = sV + st * kTileBytes + c * kPanelBytes;
@@ -331,11 +337,11 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       // Drain: every load issued here has landed before the CTA exits
       // (immediate on the normal path; bounded on the abort path).
       volatile int no_abort = 0;
-      mbar_wait(bar(kBarQ), 0, &no_abort, p.status);
+      mbar_wait(bar(kBarQ), 0, &no_abort, nullptr);
       for (int j = max(0, issued_k - kStages); j < issued_k; ++j)
-        mbar_wait(bar(kBarKFull + j % kStages), (j / kStages) & 1, &no_abort, p.status);
+        mbar_wait(bar(kBarKFull + j % kStages), (j / kStages) & 1, &no_abort, nullptr);
       for (int j = max(0, issued_v - kStages); j < issued_v; ++j)
-        mbar_wait(bar(kBarVFull + j % kStages), (j / kStages) & 1, &no_abort, p.status);
+        mbar_wait(bar(kBarVFull + j % kStages), (j / kStages) & 1, &no_abort, nullptr);
     } else if (warp == 1 && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
       constexpr uint32_t idesc_s = idesc_bf16_f32(kBlockM, kBlockN, false, false);
@@ -356,14 +362,14 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           mma_bf16_ts(tmem + 256 + x * D, tmem + x * kBlockN + kk * 8, b, idesc_o, (!first || kk > 0) ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(bar(kBarQ), 0, abort_flag, p.status);
+      bool ok = mbar_wait(bar(kBarQ), 0, abort_flag, p.status, p.wait_limit_ns);
       for (int j = 0; ok && j < n; ++j) {
         const int st = j % kStages, pst = (j + kStages - 1) % kStages;
-        if (!(ok = mbar_wait(bar(kBarKFull + st), (j / kStages) & 1, abort_flag, p.status))) break;
-        if (j > 0 && !(ok = mbar_wait(bar(kBarVFull + pst), ((j - 1) / kStages) & 1, abort_flag, p.status))) break;
+        if (!(ok = mbar_wait(bar(kBarKFull + st), (j / kStages) & 1, abort_flag, p.status, p.wait_limit_ns))) break;
+        if (j > 0 && !(ok = mbar_wait(bar(kBarVFull + pst), ((j - 1) / kStages) & 1, abort_flag, p.status, p.wait_limit_ns))) break;
         for (int x = 0; x < n_act; ++x) {
           if (j > 0) {
-            if (!(ok = mbar_wait(bar(kBarPFull + x), (j - 1) & 1, abort_flag, p.status))) break;
+            if (!(ok = mbar_wait(bar(kBarPFull + x), (j - 1) & 1, abort_flag, p.status, p.wait_limit_ns))) break;
             tc_fence_after();
             issue_pv(x, pst, j == 1);
           } else {
@@ -378,9 +384,9 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       }
       if (ok && n > 0) {
         const int pst = (n - 1) % kStages;
-        ok = mbar_wait(bar(kBarVFull + pst), ((n - 1) / kStages) & 1, abort_flag, p.status);
+        ok = mbar_wait(bar(kBarVFull + pst), ((n - 1) / kStages) & 1, abort_flag, p.status, p.wait_limit_ns);
         for (int x = 0; ok && x < n_act; ++x) {
-          if (!(ok = mbar_wait(bar(kBarPFull + x), (n - 1) & 1, abort_flag, p.status))) break;
+          if (!(ok = mbar_wait(bar(kBarPFull + x), (n - 1) & 1, abort_flag, p.status, p.wait_limit_ns))) break;
           tc_fence_after();
           issue_pv(x, pst, n == 1);
           mma_commit(bar(kBarODone + x));
@@ -389,7 +395,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       // Drain: all MMAs of this thread complete before TMEM is released.
       mma_commit(bar(kBarDrain));
       volatile int no_abort = 0;
-      mbar_wait(bar(kBarDrain), 0, &no_abort, p.status);
+      mbar_wait(bar(kBarDrain), 0, &no_abort, nullptr);
     }
   } else {
     setmaxnreg_inc224();
@@ -429,7 +435,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       const int seg_scale = int((d >> 8) & 0xFFu);
       // the tile's 128 threads agree on continuing (a per-column table and a
       // named barrier may follow)
-      ok = bar_and(3 + x, kBlockM, mbar_wait(bar(kBarSFull + x), j & 1, abort_flag, p.status));
+      ok = bar_and(3 + x, kBlockM, mbar_wait(bar(kBarSFull + x), j & 1, abort_flag, p.status, p.wait_limit_ns));
       if (!ok) break;
       tc_fence_after();
       float sv[kBlockN];
@@ -579,7 +585,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     }
 
     // ---------------------------------------------------------- epilogue
-    if (ok && n > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarODone + x), 0, abort_flag, p.status));
+    if (ok && n > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarODone + x), 0, abort_flag, p.status, p.wait_limit_ns));
     const bool row_ok = ok && r < it.rows_valid[x];
     const float inv_l = 1.f / l_sum;
     if (ok && p.out != nullptr) {
@@ -663,9 +669,27 @@ static int build_qtiles(Params& p, int query_scale) {
   return VARK_OK;
 }
 
+// Failure-detection test hook: VARK_TEST_WAIT_LIMIT_MS shortens the bounded
+// waits, VARK_TEST_WITHHOLD_KV_TILE=j makes every CTA's producer stop before
+// key tile j so the waits on it run out (the kernel then reports
+// VARK_E_TIMEOUT through the status word).  Both unset in normal use.
+static void apply_test_hooks(Params& p) {
+  p.wait_limit_ns = kWaitLimitNs;
+  p.withhold_tile = -1;
+  if (const char* e = std::getenv("VARK_TEST_WAIT_LIMIT_MS")) {
+    const long ms = std::strtol(e, nullptr, 10);
+    if (ms > 0 && ms <= 10000) p.wait_limit_ns = uint64_t(ms) * 1000000ull;
+  }
+  if (const char* e = std::getenv("VARK_TEST_WITHHOLD_KV_TILE")) {
+    const long j = std::strtol(e, nullptr, 10);
+    if (j >= 0 && j < (1 << 20)) p.withhold_tile = int(j);
+  }
+}
+
 template <int D, bool PRUNED, bool MASS>
 static int launch(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& kc,
-                  const CUtensorMap& vc, const Params& p, cudaStream_t st) {
+                  const CUtensorMap& vc, Params& p, cudaStream_t st) {
+  apply_test_hooks(p);
   auto kern = attn_kernel<D, PRUNED, MASS>;
   const int smem = Smem<D>::alloc(MASS, p.sc.S);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {

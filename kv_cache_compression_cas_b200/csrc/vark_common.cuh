@@ -50,7 +50,8 @@ int encode_bf16_map(CUtensorMap* map, const void* base, int rank, const uint64_t
 // ---------------------------------------------------------------- device side
 #define VARK_DEV __device__ __forceinline__
 
-// Bounded waits give up after this many nanoseconds of %globaltimer.
+// Bounded waits give up after this many nanoseconds of %globaltimer (the
+// attention kernels take the limit from their parameters; this is the default).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
 VARK_DEV uint32_t smem_u32(const void* p) {
@@ -113,7 +114,8 @@ VARK_DEV bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity) {
 // kWaitLimitNs: sets *abort_flag (shared) and the caller's status word, and
 // returns false.  Also returns false at once when another role has aborted
 // or another CTA of the launch has recorded an error.
-VARK_DEV bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int32_t* status) {
+VARK_DEV bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int32_t* status,
+                        uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (;;) {
@@ -123,7 +125,7 @@ VARK_DEV bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
       *abort_flag = 1;
       return false;
     }
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       *abort_flag = 1;
       if (status) atomicExch(status, VARK_E_TIMEOUT);
       return false;
