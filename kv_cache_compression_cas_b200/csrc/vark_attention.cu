@@ -286,6 +286,36 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     mbar_init(bar(kBarDrain), 1);
     *abort_flag = 0;
     fence_barrier_init();
+    // Start the first loads now, so their latency overlaps TMEM allocation
+    // and the table setup below (the producer loop continues after them).
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    if (PRUNED) {
+      tma_prefetch_desc(&tm_kc);
+      tma_prefetch_desc(&tm_vc);
+    }
+    const int qrow = (p.q_scale_rows ? 0 : p.sc.off[it.k]) + it.row0;
+    mbar_arrive_expect_tx(bar(kBarQ), n_act * kTileBytes);
+    for (int x = 0; x < n_act; ++x)
+      for (int c = 0; c < QP; ++c)
+        tma_load_3d(sQ + x * kTileBytes + c * kPanelBytes, &tm_q, bar(kBarQ), c * 64, qrow + x * kBlockM, it.bh);
+    const int first = min(min(n, kStages), p.withhold_tile < 0 ? n : p.withhold_tile);
+    for (int j = 0; j < first; ++j) {
+      const KTile t = it.tile(p, j);
+      mbar_arrive_expect_tx(bar(kBarKFull + j), kTileBytes);
+      for (int c = 0; c < QP; ++c) {
+        const uint32_t dst = sK + j * kTileBytes + c * kPanelBytes;
+        if (t.src == 0) tma_load_3d(dst, &tm_k, bar(kBarKFull + j), c * 64, t.row, it.bh);
+        else tma_load_2d(dst, &tm_kc, bar(kBarKFull + j), c * 64, t.row);
+      }
+      mbar_arrive_expect_tx(bar(kBarVFull + j), kTileBytes);
+      for (int c = 0; c < QP; ++c) {
+        const uint32_t dst = sV + j * kTileBytes + c * kPanelBytes;
+        if (t.src == 0) tma_load_3d(dst, &tm_v, bar(kBarVFull + j), c * 64, t.row, it.bh);
+        else tma_load_2d(dst, &tm_vc, bar(kBarVFull + j), c * 64, t.row);
+      }
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -300,20 +330,11 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     setmaxnreg_dec56();
     if (warp == 0 && lane == 0) {
       // ---------------------------------------------------------- producer
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      if (PRUNED) {
-        tma_prefetch_desc(&tm_kc);
-        tma_prefetch_desc(&tm_vc);
-      }
-      const int qrow = (p.q_scale_rows ? 0 : p.sc.off[it.k]) + it.row0;
-      mbar_arrive_expect_tx(bar(kBarQ), n_act * kTileBytes);
-      for (int x = 0; x < n_act; ++x)
-        for (int c = 0; c < QP; ++c)
-          tma_load_3d(sQ + x * kTileBytes + c * kPanelBytes, &tm_q, bar(kBarQ), c * 64, qrow + x * kBlockM, it.bh);
-      int issued_k = 0, issued_v = 0;
-      for (int j = 0; j < n; ++j) {
+      // (Q and the first kStages key tiles were issued right after the
+      // barrier initialisation, by this same thread.)
+      int issued_k = min(min(n, kStages), p.withhold_tile < 0 ? n : p.withhold_tile);
+      int issued_v = issued_k;
+      for (int j = issued_k; j < n; ++j) {
         const int st = j % kStages;
         const KTile t = it.tile(p, j);
         if (j == p.withhold_tile) break;   // test hook: this tile never arrives
@@ -614,11 +635,21 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     if (MASS) {
       // mean over the B * n_k rows of scale k of m_i(s): both tiles' rows are
       // reduced in the CTA, then one atomic per (h, s, k)
-      for (int s = 0; s <= it.k; ++s) {
-        float v = row_ok ? mrow[s * kBlockM] * inv_l : 0.f;
+      for (int s0 = 0; s0 <= it.k; s0 += 16) {
+        float v[16];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) red_sm[(x * 4 + (warp & 3)) * 32 + s] = v;
+        for (int i = 0; i < 16; ++i) v[i] = (row_ok && s0 + i <= it.k) ? mrow[(s0 + i) * kBlockM] * inv_l : 0.f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] += __shfl_xor_sync(0xffffffffu, v[i], o);
+        }
+        if (lane < 16 && s0 + lane <= it.k) {
+          float mine = v[0];
+#pragma unroll
+          for (int i = 1; i < 16; ++i) mine = (lane == i) ? v[i] : mine;
+          red_sm[(x * 4 + (warp & 3)) * 32 + s0 + lane] = mine;
+        }
       }
       named_bar_sync(1, 2 * kBlockM);
       if (x == 0 && r <= it.k && *abort_flag == 0) {
