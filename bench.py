@@ -59,6 +59,24 @@ def _peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def measured_traffic():
+    """DRAM bytes per full calibration launch from the committed ncu summary,
+    or None when the attention kernel's source has changed since the capture."""
+    import hashlib
+    import re
+    prof = os.path.join(ROOT, "profiles", "attn_calib_1024_4seeds_16heads.md")
+    src = os.path.join(ROOT, "kv_cache_compression_cas_b200", "csrc", "vark_attention.cu")
+    try:
+        text = open(prof).read()
+        m = re.search(r"Traffic per full launch \(bytes\): (\d+) \(kernel ([0-9a-f]+)\)", text)
+        cur = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    if not m or m.group(2) != cur:
+        return None
+    return int(m.group(1))
+
+
 # ---------------------------------------------------------------- algorithmic work
 def calib_flops(sides, B, H, D):
     n = [s * s for s in sides]
@@ -468,7 +486,8 @@ def main():
     per_launch_s = ph["calib"] / (K * L)
     roof = {"bound": "tensor", "kernel": "attn_kernel<128,false,true> (S-CAS calibration attention)",
             "achieved": per_launch_flops / per_launch_s / 1e12, "peak": peaks["bf16_tflops_sustained"],
-            "unit": "TFLOP/s", "traffic": None,
+            "unit": "TFLOP/s", "traffic": measured_traffic(),
+            "traffic_source": "profiles/attn_calib_1024_4seeds_16heads.md (ncu dram bytes of a 4-seed launch x 4)",
             "peak_kind": f"bf16 dense sustained ({peaks['source']})"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     kernels = {
