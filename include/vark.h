@@ -209,6 +209,66 @@ int vark_pruned_attention(const uint16_t* q, const uint16_t* kc, const uint16_t*
                           const float* tau, const float* bias,
                           uint16_t* out, int32_t* dev_status, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Generation order.  [HeatKV] Method step 5: the static schedule keeps cache use
+ * within budget as new scales are generated.  Scale k is generated, its queries
+ * attend to the cache built so far plus scale k itself, then scale k's retained
+ * blocks are appended to the compacted cache.  The compacted buffers use the
+ * final layout of vark_build_offsets from the start (every segment has its
+ * final place); rows that no append has written yet must hold finite values,
+ * so zero-initialise kc / vc once before the first scale.
+ * ------------------------------------------------------------------------- */
+
+/*
+ * vark_append_scale -- device.  Appends scale `scale` of every layer: for each
+ * (l, b, h) with keep[l][h][scale], copies the n_k rows of the new scale's K and
+ * V to row b*R_l + head_off[l][h] + seg_off[l][h][scale] of layer l's block.
+ *   k_new, v_new  dev bf16, layer l's new-scale block [B][H][n_k][D] at element
+ *                 l * layer_stride (layer_stride >= B*H*n_k*D).
+ *   other arguments as vark_compact_kv.
+ * Appending scales 0..S-1 in turn leaves kc / vc equal to vark_compact_kv's.
+ * Errors: VARK_E_ARG, VARK_E_SHAPE, VARK_E_ALIGN, VARK_E_CUDA.
+ */
+int vark_append_scale(const uint16_t* k_new, const uint16_t* v_new, int64_t layer_stride,
+                      int L, int B, int H, int S, int D, const int32_t* sides, int scale,
+                      const uint8_t* keep, const int32_t* head_off, const int32_t* seg_off,
+                      const int64_t* layer_base, uint16_t* kc, uint16_t* vc, void* stream);
+
+/*
+ * vark_pruned_attention_step -- device.  Pruned attention of one layer for the
+ * queries of scale `scale` while that scale is generated: keys = the head's
+ * retained past scales s < scale (compacted, past_len[h][scale] rows) followed
+ * by the n_k rows of the new scale itself ([AMS-KV] Abstract: the local scale
+ * is always attended).  Identical arithmetic to vark_pruned_attention with
+ * query_scale = scale; only the local scale's K / V come as their own block.
+ *   q            dev bf16 [B][H][n_k][D]
+ *   k_local, v_local  dev bf16 [B][H][n_k][D], the new scale's keys / values
+ *   out          dev bf16 [B][H][n_k][D]
+ *   other arguments as vark_pruned_attention.
+ * Errors: as vark_pruned_attention.
+ */
+int vark_pruned_attention_step(const uint16_t* q, const uint16_t* kc, const uint16_t* vc, int64_t kc_rows,
+                               const uint16_t* k_local, const uint16_t* v_local,
+                               int B, int H, int S, int D, const int32_t* sides, int scale,
+                               const int32_t* head_off, const int32_t* seg_off, const int32_t* past_len,
+                               const float* tau, const float* bias,
+                               uint16_t* out, int32_t* dev_status, void* stream);
+
+/*
+ * vark_cache_size_after_layer -- host.  Cache-size accounting while scales are
+ * generated ([Review] Appendix A, Algorithm 2 CACHESIZEAFTERLAYER(k, l, G_k,
+ * G_k-1, E_k); its body is truncated on the page).  Reading for a static
+ * schedule (G_k = G_k-1 = the dropped pairs, E_k = scale k's entries): during
+ * scale k the layers run in order, so after layer l the layers 0..l hold their
+ * retained scales <= k and the layers l+1.. their retained scales < k.
+ *   bytes  host int64 [S][L]: bytes[k][l] = retained K + V bytes (bf16) held
+ *          after layer l during scale k; bytes[S-1][L-1] = 2 * 2 * layer_base[L].
+ *   keep   host uint8 [L][H][S].
+ * Errors: VARK_E_ARG, VARK_E_SHAPE.
+ */
+int vark_cache_size_after_layer(const uint8_t* keep, int L, int H, int S, const int32_t* sides, int B, int D,
+                                int64_t* bytes);
+
 #ifdef __cplusplus
 }
 #endif

@@ -47,6 +47,10 @@ _SIGNATURES = {
     "vark_compact_kv": (_I, [_P, _P, _I64, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
     "vark_pruned_attention": (_I, [_P, _P, _P, _I64, _P, _P, _I, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P, _P,
                                    _P, _P]),
+    "vark_pruned_attention_step": (_I, [_P, _P, _P, _I64, _P, _P, _I, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P,
+                                        _P, _P, _P]),
+    "vark_append_scale": (_I, [_P, _P, _I64, _I, _I, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P, _P, _P]),
+    "vark_cache_size_after_layer": (_I, [_P, _I, _I, _I, _P, _I, _I, _P]),
 }
 
 
@@ -200,3 +204,50 @@ def vark_pruned_attention(q, kc, vc, kc_rows: int, k_dense, v_dense, sides, quer
         _dptr(bias, torch.float32, "bias"), _dptr(out, torch.bfloat16, "out"),
         _dptr(dev_status, torch.int32, "dev_status"), _stream(stream))
     _check(rc, "vark_pruned_attention")
+
+
+def vark_append_scale(k_new, v_new, layer_stride: int, L: int, B: int, H: int, sides, D: int, scale: int, keep,
+                      head_off, seg_off, layer_base, kc, vc, stream=None):
+    """Device: append scale `scale` of every layer to the compacted cache."""
+    import torch
+    s_arr, s_ptr = _sides_arg(sides)
+    rc = _load().vark_append_scale(
+        _dptr(k_new, torch.bfloat16, "k_new"), _dptr(v_new, torch.bfloat16, "v_new"), int(layer_stride), int(L),
+        int(B), int(H), len(s_arr), int(D), s_ptr, int(scale), _dptr(keep, torch.uint8, "keep"),
+        _dptr(head_off, torch.int32, "head_off"), _dptr(seg_off, torch.int32, "seg_off"),
+        _dptr(layer_base, torch.int64, "layer_base"), _dptr(kc, torch.bfloat16, "kc"),
+        _dptr(vc, torch.bfloat16, "vc"), _stream(stream))
+    _check(rc, "vark_append_scale")
+
+
+def vark_pruned_attention_step(q, kc, vc, kc_rows: int, k_local, v_local, sides, scale: int, head_off, seg_off,
+                               past_len, tau, bias, out, dev_status, stream=None):
+    """Device: pruned attention for the queries of the scale being generated."""
+    import torch
+    B, H, _, D = k_local.shape
+    s_arr, s_ptr = _sides_arg(sides)
+    kcp = kc.data_ptr() if (kc is not None and kc_rows > 0) else None
+    vcp = vc.data_ptr() if (vc is not None and kc_rows > 0) else None
+    if kc is not None:
+        _dptr(kc, torch.bfloat16, "kc")
+        _dptr(vc, torch.bfloat16, "vc")
+    rc = _load().vark_pruned_attention_step(
+        _dptr(q, torch.bfloat16, "q"), kcp, vcp, int(kc_rows),
+        _dptr(k_local, torch.bfloat16, "k_local"), _dptr(v_local, torch.bfloat16, "v_local"),
+        int(B), int(H), len(s_arr), int(D), s_ptr, int(scale),
+        _dptr(head_off, torch.int32, "head_off"), _dptr(seg_off, torch.int32, "seg_off"),
+        _dptr(past_len, torch.int32, "past_len"), _dptr(tau, torch.float32, "tau"),
+        _dptr(bias, torch.float32, "bias"), _dptr(out, torch.bfloat16, "out"),
+        _dptr(dev_status, torch.int32, "dev_status"), _stream(stream))
+    _check(rc, "vark_pruned_attention_step")
+
+
+def vark_cache_size_after_layer(keep: np.ndarray, sides, B: int, D: int) -> np.ndarray:
+    """Host: int64 [S][L] retained K+V bytes after layer l during scale k."""
+    kp = np.ascontiguousarray(keep, dtype=np.uint8)
+    L, H, S = kp.shape
+    s_arr, s_ptr = _sides_arg(sides)
+    out = np.zeros((S, L), dtype=np.int64)
+    _check(_load().vark_cache_size_after_layer(kp.ctypes.data, L, H, S, s_ptr, int(B), int(D), out.ctypes.data),
+           "vark_cache_size_after_layer")
+    return out

@@ -72,6 +72,7 @@ struct Params {
   int32_t* status;
   int q_rows;                     // rows per (b, h) of q / out
   int q_scale_rows;               // 1: q row = row within scale (single-scale q)
+  int local_scale_only;           // 1: the local K/V source holds only the query scale's rows
   // pruned attention
   int64_t R_l;
   const int32_t* head_off;        // [H]
@@ -147,7 +148,7 @@ struct Item {
     } else {
       const int jj = j - n_past;
       t.src = 0;
-      t.row = p.sc.off[k] + jj * kBlockN;
+      t.row = (p.local_scale_only ? 0 : p.sc.off[k]) + jj * kBlockN;
       t.valid = min(kBlockN, p.sc.n[k] - jj * kBlockN);
       t.key0 = jj * kBlockN;
     }
@@ -757,7 +758,7 @@ extern "C" int vark_scas_accumulate(const uint16_t* q, const uint16_t* k, const 
   lp.B = B; lp.H = H;
   lp.scale_log2 = kLog2e / sqrtf(float(D));
   lp.tau = tau; lp.bias = bias; lp.mass = mass; lp.out = out; lp.status = dev_status;
-  lp.q_rows = lp.sc.T; lp.q_scale_rows = 0;
+  lp.q_rows = lp.sc.T; lp.q_scale_rows = 0; lp.local_scale_only = 0;
   lp.R_l = 0; lp.head_off = nullptr; lp.seg_off = nullptr; lp.past_len = nullptr;
   if ((rc = build_qtiles(lp, -1))) return rc;
   CUtensorMap tq, tk, tv;
@@ -769,22 +770,22 @@ extern "C" int vark_scas_accumulate(const uint16_t* q, const uint16_t* k, const 
                   : launch<64, false, true>(tq, tk, tv, tk, tv, lp, st);
 }
 
-extern "C" int vark_pruned_attention(const uint16_t* q, const uint16_t* kc, const uint16_t* vc, int64_t kc_rows,
-                                     const uint16_t* k_dense, const uint16_t* v_dense, int B, int H, int S, int D,
-                                     const int32_t* sides, int query_scale, const int32_t* head_off,
-                                     const int32_t* seg_off, const int32_t* past_len, const float* tau,
-                                     const float* bias, uint16_t* out, int32_t* dev_status, void* stream) {
-  if (!q || !k_dense || !v_dense || !head_off || !seg_off || !past_len || !tau || !out || !dev_status)
+static int pruned_common(const uint16_t* q, const uint16_t* kc, const uint16_t* vc, int64_t kc_rows,
+                         const uint16_t* k_local, const uint16_t* v_local, int B, int H, int S, int D,
+                         const int32_t* sides, int query_scale, bool local_scale_only, const int32_t* head_off,
+                         const int32_t* seg_off, const int32_t* past_len, const float* tau, const float* bias,
+                         uint16_t* out, int32_t* dev_status, void* stream) {
+  if (!q || !k_local || !v_local || !head_off || !seg_off || !past_len || !tau || !out || !dev_status)
     return VARK_E_ARG;
   if (kc_rows < 0 || (kc_rows > 0 && (!kc || !vc))) return VARK_E_ARG;
   Params lp;
   int rc = make_scale_table(S, sides, &lp.sc);
   if (rc) return rc;
   if (D != 64 && D != 128) return VARK_E_SHAPE;
-  if (query_scale < -1 || query_scale >= S) return VARK_E_ARG;
+  if (query_scale < -1 || query_scale >= S || (local_scale_only && query_scale < 0)) return VARK_E_ARG;
   if (!finite_shape(B, H, lp.sc.T, D)) return VARK_E_SHAPE;
   if (kc_rows % B != 0 || kc_rows > INT32_MAX) return VARK_E_SHAPE;
-  if (!aligned16(q) || !aligned16(k_dense) || !aligned16(v_dense) || !aligned16(out) ||
+  if (!aligned16(q) || !aligned16(k_local) || !aligned16(v_local) || !aligned16(out) ||
       (kc_rows > 0 && (!aligned16(kc) || !aligned16(vc))))
     return VARK_E_ALIGN;
   if ((rc = check_device_sm100())) return rc;
@@ -793,23 +794,45 @@ extern "C" int vark_pruned_attention(const uint16_t* q, const uint16_t* kc, cons
   lp.tau = tau; lp.bias = bias; lp.mass = nullptr; lp.out = out; lp.status = dev_status;
   lp.q_rows = query_scale < 0 ? lp.sc.T : lp.sc.n[query_scale];
   lp.q_scale_rows = query_scale < 0 ? 0 : 1;
+  lp.local_scale_only = local_scale_only ? 1 : 0;
   lp.R_l = kc_rows / B;
   lp.head_off = head_off; lp.seg_off = seg_off; lp.past_len = past_len;
   if ((rc = build_qtiles(lp, query_scale))) return rc;
+  const int64_t local_rows = local_scale_only ? lp.sc.n[query_scale] : lp.sc.T;
   CUtensorMap tq, tk, tv, tkc, tvc;
   if ((rc = encode_dense(&tq, q, D, lp.q_rows, int64_t(B) * H))) return rc;
-  if ((rc = encode_dense(&tk, k_dense, D, lp.sc.T, int64_t(B) * H))) return rc;
-  if ((rc = encode_dense(&tv, v_dense, D, lp.sc.T, int64_t(B) * H))) return rc;
+  if ((rc = encode_dense(&tk, k_local, D, local_rows, int64_t(B) * H))) return rc;
+  if ((rc = encode_dense(&tv, v_local, D, local_rows, int64_t(B) * H))) return rc;
   if (kc_rows > 0) {
     if ((rc = encode_rows(&tkc, kc, D, kc_rows))) return rc;
     if ((rc = encode_rows(&tvc, vc, D, kc_rows))) return rc;
   } else {
     // No head keeps past rows, so these maps are never read; they only need
     // to be valid 2-D maps.
-    if ((rc = encode_rows(&tkc, k_dense, D, 1))) return rc;
-    if ((rc = encode_rows(&tvc, v_dense, D, 1))) return rc;
+    if ((rc = encode_rows(&tkc, k_local, D, 1))) return rc;
+    if ((rc = encode_rows(&tvc, v_local, D, 1))) return rc;
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return D == 128 ? launch<128, true, false>(tq, tk, tv, tkc, tvc, lp, st)
                   : launch<64, true, false>(tq, tk, tv, tkc, tvc, lp, st);
+}
+
+extern "C" int vark_pruned_attention(const uint16_t* q, const uint16_t* kc, const uint16_t* vc, int64_t kc_rows,
+                                     const uint16_t* k_dense, const uint16_t* v_dense, int B, int H, int S, int D,
+                                     const int32_t* sides, int query_scale, const int32_t* head_off,
+                                     const int32_t* seg_off, const int32_t* past_len, const float* tau,
+                                     const float* bias, uint16_t* out, int32_t* dev_status, void* stream) {
+  return pruned_common(q, kc, vc, kc_rows, k_dense, v_dense, B, H, S, D, sides, query_scale, false, head_off,
+                       seg_off, past_len, tau, bias, out, dev_status, stream);
+}
+
+extern "C" int vark_pruned_attention_step(const uint16_t* q, const uint16_t* kc, const uint16_t* vc,
+                                          int64_t kc_rows, const uint16_t* k_local, const uint16_t* v_local, int B,
+                                          int H, int S, int D, const int32_t* sides, int scale,
+                                          const int32_t* head_off, const int32_t* seg_off, const int32_t* past_len,
+                                          const float* tau, const float* bias, uint16_t* out, int32_t* dev_status,
+                                          void* stream) {
+  if (scale < 0) return VARK_E_ARG;
+  return pruned_common(q, kc, vc, kc_rows, k_local, v_local, B, H, S, D, sides, scale, true, head_off, seg_off,
+                       past_len, tau, bias, out, dev_status, stream);
 }

@@ -110,3 +110,23 @@ extern "C" int vark_build_schedule(const double* scas, int L, int H, int S, cons
   }
   return VARK_OK;
 }
+
+extern "C" int vark_cache_size_after_layer(const uint8_t* keep, int L, int H, int S, const int32_t* sides, int B,
+                                           int D, int64_t* bytes) {
+  if (keep == nullptr || bytes == nullptr || sides == nullptr) return VARK_E_ARG;
+  int64_t T = 0;
+  if (L < 1 || H < 1 || B < 1 || D < 1 || !sides_ok(S, sides, &T)) return VARK_E_SHAPE;
+  int64_t total = 0;
+  const int64_t per_token = int64_t(B) * D * 2 * 2;   // K and V, bf16
+  for (int k = 0; k < S; ++k) {
+    const int64_t n = int64_t(sides[k]) * sides[k];
+    for (int l = 0; l < L; ++l) {
+      int64_t kept_heads = 0;
+      for (int h = 0; h < H; ++h) kept_heads += keep[(int64_t(l) * H + h) * S + k] ? 1 : 0;
+      const int64_t add = kept_heads * n * per_token;
+      total += add;
+      bytes[int64_t(k) * L + l] = total;
+    }
+  }
+  return VARK_OK;
+}

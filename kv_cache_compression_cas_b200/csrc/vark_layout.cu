@@ -73,10 +73,12 @@ constexpr int kMaxGroupLH = 4096;   // (layer, head) pairs per launch group
 
 struct CompactParams {
   ScaleTable sc;
-  int32_t chunks[VARK_MAX_SCALES];  // ceil(n_s / kChunkRows)
+  int32_t chunks[VARK_MAX_SCALES];  // ceil(n_s / kChunkRows) for scales in [s_lo, s_hi), else 0
+  int32_t src_off[VARK_MAX_SCALES]; // first source row of scale s inside a (b, h) block of the source
+  int64_t src_rows;                 // rows per (b, h) block of the source (T, or n_k for one scale)
   int l0, nl;                       // layer group [l0, l0 + nl)
   int L, B, H, D;
-  int64_t layer_stride;             // elements between dense layers
+  int64_t layer_stride;             // elements between source layers
 };
 
 __global__ void __launch_bounds__(kCompactThreads) compact_kernel(
@@ -98,7 +100,7 @@ __global__ void __launch_bounds__(kCompactThreads) compact_kernel(
     uint32_t m = 0;
     int32_t c = 0;
     for (int s = 0; s < S; ++s) {
-      if (kp[s]) {
+      if (kp[s] && p.chunks[s] > 0) {
         m |= 1u << s;
         c += p.chunks[s];
       }
@@ -141,7 +143,6 @@ __global__ void __launch_bounds__(kCompactThreads) compact_kernel(
 
   const int64_t units = int64_t(grand) * p.B;
   const int vec_per_row = p.D / 8;  // 16-byte vectors per row
-  const int64_t T = p.sc.T;
 
   for (int64_t g = blockIdx.x; g < units; g += gridDim.x) {
     const int b = int(g % p.B);
@@ -168,7 +169,7 @@ __global__ void __launch_bounds__(kCompactThreads) compact_kernel(
     const int32_t nrows = min(kChunkRows, p.sc.n[s] - r0);
     const int64_t R_l = (layer_base[l + 1] - layer_base[l]) / (int64_t(p.B) * p.D);
     const int64_t dst_row = int64_t(b) * R_l + head_off[l * H + h] + seg_off[(l * H + h) * S + s] + r0;
-    const int64_t src_row = (int64_t(b) * H + h) * T + p.sc.off[s] + r0;
+    const int64_t src_row = (int64_t(b) * H + h) * p.src_rows + p.src_off[s] + r0;
     const int64_t dst_v = (layer_base[l] / 8) + dst_row * vec_per_row;
     const int64_t src_v = (int64_t(l) * p.layer_stride) / 8 + src_row * vec_per_row;
     const int nvec = nrows * vec_per_row;
@@ -218,6 +219,34 @@ extern "C" int vark_build_offsets(const uint8_t* keep, int L, int H, int S, cons
   return cudaGetLastError() == cudaSuccess ? VARK_OK : VARK_E_CUDA;
 }
 
+// Launches the gather for scales [s_lo, s_hi) of a source laid out per layer
+// as [B][H][src_rows][D] with scale s starting at row src_off[s].
+static int launch_gather(const uint16_t* k, const uint16_t* v, int64_t layer_stride, int L, int B, int H, int D,
+                         CompactParams& p, int s_lo, int s_hi, int64_t src_rows, const int32_t* src_off,
+                         const uint8_t* keep, const int32_t* head_off, const int32_t* seg_off,
+                         const int64_t* layer_base, uint16_t* kc, uint16_t* vc, cudaStream_t st) {
+  p.L = L; p.B = B; p.H = H; p.D = D; p.layer_stride = layer_stride; p.src_rows = src_rows;
+  for (int s = 0; s < VARK_MAX_SCALES; ++s) {
+    const bool in = s < p.sc.S && s >= s_lo && s < s_hi;
+    p.chunks[s] = in ? (p.sc.n[s] + kChunkRows - 1) / kChunkRows : 0;
+    p.src_off[s] = in ? src_off[s] : 0;
+  }
+  int dev = 0, nsm = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  const int layers_per_group = std::max(1, kMaxGroupLH / H);
+  for (int l0 = 0; l0 < L; l0 += layers_per_group) {
+    p.l0 = l0;
+    p.nl = std::min(layers_per_group, L - l0);
+    compact_kernel<<<nsm * 4, kCompactThreads, 0, st>>>(reinterpret_cast<const uint4*>(k),
+                                                        reinterpret_cast<const uint4*>(v), p, keep, head_off,
+                                                        seg_off, layer_base, reinterpret_cast<uint4*>(kc),
+                                                        reinterpret_cast<uint4*>(vc));
+    if (cudaGetLastError() != cudaSuccess) return VARK_E_CUDA;
+  }
+  return VARK_OK;
+}
+
 extern "C" int vark_compact_kv(const uint16_t* k, const uint16_t* v, int64_t layer_stride, int L, int B, int H,
                                int S, int D, const int32_t* sides, const uint8_t* keep, const int32_t* head_off,
                                const int32_t* seg_off, const int64_t* layer_base, uint16_t* kc, uint16_t* vc,
@@ -232,22 +261,26 @@ extern "C" int vark_compact_kv(const uint16_t* k, const uint16_t* v, int64_t lay
   if (layer_stride % 8 != 0) return VARK_E_ALIGN;
   if (!aligned16(k) || !aligned16(v) || !aligned16(kc) || !aligned16(vc)) return VARK_E_ALIGN;
   if ((rc = check_device_sm100())) return rc;
-  p.L = L; p.B = B; p.H = H; p.D = D; p.layer_stride = layer_stride;
-  for (int s = 0; s < VARK_MAX_SCALES; ++s)
-    p.chunks[s] = s < S ? (p.sc.n[s] + kChunkRows - 1) / kChunkRows : 0;
-  int dev = 0, nsm = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  const int layers_per_group = std::max(1, kMaxGroupLH / H);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  for (int l0 = 0; l0 < L; l0 += layers_per_group) {
-    p.l0 = l0;
-    p.nl = std::min(layers_per_group, L - l0);
-    compact_kernel<<<nsm * 4, kCompactThreads, 0, st>>>(reinterpret_cast<const uint4*>(k),
-                                                        reinterpret_cast<const uint4*>(v), p, keep, head_off,
-                                                        seg_off, layer_base, reinterpret_cast<uint4*>(kc),
-                                                        reinterpret_cast<uint4*>(vc));
-    if (cudaGetLastError() != cudaSuccess) return VARK_E_CUDA;
-  }
-  return VARK_OK;
+  return launch_gather(k, v, layer_stride, L, B, H, D, p, 0, S, p.sc.T, p.sc.off, keep, head_off, seg_off,
+                       layer_base, kc, vc, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int vark_append_scale(const uint16_t* k_new, const uint16_t* v_new, int64_t layer_stride, int L, int B,
+                                 int H, int S, int D, const int32_t* sides, int scale, const uint8_t* keep,
+                                 const int32_t* head_off, const int32_t* seg_off, const int64_t* layer_base,
+                                 uint16_t* kc, uint16_t* vc, void* stream) {
+  if (!k_new || !v_new || !keep || !head_off || !seg_off || !layer_base || !kc || !vc) return VARK_E_ARG;
+  CompactParams p;
+  int rc = make_scale_table(S, sides, &p.sc);
+  if (rc) return rc;
+  if (scale < 0 || scale >= S) return VARK_E_ARG;
+  if (L < 1 || H < 1 || B < 1 || D < 8 || D % 8 != 0 || D > 1024) return VARK_E_SHAPE;
+  if (H > kMaxGroupLH) return VARK_E_SHAPE;
+  if (layer_stride < int64_t(B) * H * p.sc.n[scale] * D) return VARK_E_ARG;
+  if (layer_stride % 8 != 0) return VARK_E_ALIGN;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(kc) || !aligned16(vc)) return VARK_E_ALIGN;
+  if ((rc = check_device_sm100())) return rc;
+  int32_t zero_off[VARK_MAX_SCALES] = {0};
+  return launch_gather(k_new, v_new, layer_stride, L, B, H, D, p, scale, scale + 1, p.sc.n[scale], zero_off, keep,
+                       head_off, seg_off, layer_base, kc, vc, static_cast<cudaStream_t>(stream));
 }

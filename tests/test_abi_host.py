@@ -93,3 +93,10 @@ def test_argument_errors_are_status_codes():
     assert lib.vark_compact_kv(p, p, 1 << 20, 1, 1, 4, 7, 12, sides, p, p, p, p, p, p, None) == -2
     assert lib.vark_build_offsets(p, 1, 4, 7, sides, 1, 64, None, p, p, p, None) == -1
     assert lib.vark_build_offsets(p, 1, 4, 7, sides, 1, 64, ctypes.c_void_p(20), p, p, p, None) == -3
+
+
+@pytest.mark.parametrize("sides,L,H", [(SIDES_TINY, 3, 4), (SIDES_1024, 8, 32)])
+def test_cache_size_accounting_matches_oracle(sides, L, H):
+    keep = np.random.default_rng(L + H).integers(0, 2, size=(L, H, len(sides))).astype(np.uint8)
+    got = vark.vark_cache_size_after_layer(keep, sides, 4, 128)
+    assert np.array_equal(got, oracle.cache_size_after_layer(keep, sides, 4, 128))

@@ -404,3 +404,40 @@ def _patch_transposed_scale(mp):
                                    _patch_transposed_scale])
 def test_planted_mistakes_are_caught(monkeypatch, patch):
     assert _mutant_checks(monkeypatch, patch) >= 1
+
+
+# ---------------------------------------------------------------- generation order
+
+def test_appending_every_scale_reproduces_compaction():
+    sides = SIDES_TINY
+    g = _geom(sides)
+    L, B, H, D = 2, 2, 3, 8
+    kd = normal_bf16_bits(derive_key(77, 1), (L, B, H, g.T, D))
+    vd = normal_bf16_bits(derive_key(77, 2), (L, B, H, g.T, D))
+    keep = np.random.default_rng(77).integers(0, 2, size=(L, H, g.S)).astype(np.uint8)
+    ho, so, pl, lb = oracle.build_offsets(keep, sides, B, D)
+    kref, vref = oracle.compact_kv(kd, vd, keep, sides, ho, so, lb)
+    kc = np.zeros(int(lb[-1]), dtype=np.uint16)
+    vc = np.zeros(int(lb[-1]), dtype=np.uint16)
+    for k in range(g.S):
+        sl = slice(g.off[k], g.off[k] + g.n[k])
+        oracle.append_scale(kc, vc, np.ascontiguousarray(kd[:, :, :, sl]), np.ascontiguousarray(vd[:, :, :, sl]),
+                            keep, sides, ho, so, lb, k)
+    assert np.array_equal(kc, kref) and np.array_equal(vc, vref)
+
+
+def test_cache_size_accounting_closed_forms():
+    sides = SIDES_TINY
+    g = _geom(sides)
+    L, H, B, D = 3, 4, 2, 64
+    full = np.ones((L, H, g.S), dtype=np.uint8)
+    sz = oracle.cache_size_after_layer(full, sides, B, D)
+    per = H * B * D * 4
+    for k in range(g.S):
+        for l in range(L):
+            assert sz[k, l] == L * g.off[k] * per + (l + 1) * g.n[k] * per
+    keep = np.random.default_rng(3).integers(0, 2, size=(L, H, g.S)).astype(np.uint8)
+    sz = oracle.cache_size_after_layer(keep, sides, B, D)
+    assert np.all(np.diff(sz.ravel()) >= 0)
+    _, _, _, lb = oracle.build_offsets(keep, sides, B, D)
+    assert sz[-1, -1] == 4 * int(lb[-1])
