@@ -331,6 +331,73 @@ class CpuSample:
         return flops
 
 
+def generation_order(pipe, passes, max_over_ranks, sum_over_ranks):
+    """The inference flow scale by scale on the same workload and schedule:
+    for each scale k, pruned attention of scale k's queries in every layer over
+    the cache appended so far plus scale k itself, then the append of scale k
+    for all layers.  Returns its throughput next to the one-shot path's."""
+    import torch
+    vark, w = pipe.vark, pipe.w
+    L, B, H, D = w.layers, w.batch, w.heads, w.head_dim
+    sides = pipe.sides
+    n = [s * s for s in sides]
+    off = np.cumsum([0] + n[:-1])
+    per_scale = []
+    for k in range(len(sides)):
+        sl = slice(int(off[k]), int(off[k]) + n[k])
+        per_scale.append((pipe.q[:, :, :, sl].contiguous(), pipe.k[:, :, :, sl].contiguous(),
+                          pipe.v[:, :, :, sl].contiguous()))
+    keep = pipe.last_keep
+    base = pipe.base_host.numpy()
+    st = torch.cuda.current_stream()
+    ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(2 * len(sides) * passes + 2)]
+    outs = [torch.empty_like(t[0]) for t in per_scale]
+
+    def one_pass(evs):
+        pipe.kc.zero_()
+        pipe.vc.zero_()
+        for k, (qk, kk, vk) in enumerate(per_scale):
+            if evs is not None:
+                evs[2 * k].record(st)
+            for l in range(L):
+                rows = int(base[l + 1] - base[l]) // D
+                b0, b1 = int(base[l]), int(base[l + 1])
+                vark.vark_pruned_attention_step(qk[l], pipe.kc[b0:b1] if rows else None,
+                                                pipe.vc[b0:b1] if rows else None, rows, kk[l], vk[l], sides, k,
+                                                pipe.head_off[l], pipe.seg_off[l], pipe.past_len[l], pipe.tau[l],
+                                                pipe.bias[l], outs[k][l], pipe.status)
+            if evs is not None:
+                evs[2 * k + 1].record(st)
+            vark.vark_append_scale(kk, vk, B * H * n[k] * D, L, B, H, sides, D, k, pipe.keep, pipe.head_off,
+                                   pipe.seg_off, pipe.layer_base, pipe.kc, pipe.vc)
+
+    one_pass(None)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    attn_s = 0.0
+    e0.record(st)
+    for i in range(passes):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * len(sides))]
+        one_pass(evs)
+        torch.cuda.synchronize()
+        attn_s += sum(evs[2 * k].elapsed_time(evs[2 * k + 1]) for k in range(len(sides))) / 1e3
+    e1.record(st)
+    torch.cuda.synchronize()
+    assert int(pipe.status.item()) == 0
+    t = max_over_ranks(e0.elapsed_time(e1) / 1e3)
+    attn_s = max_over_ranks(attn_s)
+    fl = pruned_flops(keep, sides, B, D) * passes
+    nl = np.array(n, dtype=np.int64)
+    kept_rows = int((keep.astype(np.int64) * nl[None, None, :]).sum())
+    app_bytes = 2.0 * kept_rows * B * D * 2 * 2 * passes
+    return {"passes": passes, "ms_per_pass": t * 1e3 / passes,
+            "attention_tflops": sum_over_ranks(fl) / attn_s / 1e12,
+            "append_and_zero_ms_per_pass": (t - attn_s) * 1e3 / passes,
+            "query_tokens_per_s": sum_over_ranks(float(L * B * pipe.T * passes)) / t,
+            "append_bytes_per_pass": app_bytes / passes,
+            "launches_per_pass": len(sides) * (L + 1) + 2}
+
+
 def reduce_over_ranks(x: float, op: str, world: int, device) -> float:
     """Max or sum of a host float over all ranks (timing plumbing; no data-path
     collective).  Works with NCCL (CUDA device) and gloo (CPU device)."""
@@ -403,6 +470,7 @@ def main():
     ap.add_argument("--impl", default="vark", choices=["vark", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--gen-passes", type=int, default=2)
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -535,6 +603,13 @@ def main():
                "d2h_bytes_per_step": d2h, "steps": ke}
         del host_in, host_out
 
+    # ------------------------------------------------ generation order (scale by scale)
+    gen = None
+    if args.gen_passes > 0:
+        del pipe.cq, pipe.ck, pipe.cv
+        torch.cuda.empty_cache()
+        gen = generation_order(pipe, args.gen_passes, max_over_ranks, sum_over_ranks)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         from threadpoolctl import threadpool_info
@@ -562,7 +637,8 @@ def main():
                        "value_def": "(calibration + pruned attention FLOPs) / step time; step = calibration, "
                                     "S-CAS, schedule, offsets, compaction, pruned attention of all layers"},
             "pruned_attention_tflops": pruned_tflops, "query_tokens_per_s": qtok_s, "compaction_gbs": comp_gbs,
-            "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+            "roofline": roof, "kernels": kernels, "generation_order": gen, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches,
             "clocks": clk, "peaks": peaks,
         }
         print(json.dumps(line), flush=True)
