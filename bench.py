@@ -331,6 +331,31 @@ class CpuSample:
         return flops
 
 
+def ranking_stability(pipe):
+    """S-CAS of every layer from two disjoint halves of the calibration seeds,
+    compared by vark_rank_stability (Spearman over candidate pairs, Jaccard of
+    the two schedules' drop sets at the workload's budget)."""
+    import torch
+    vark, w = pipe.vark, pipe.w
+    L, H, S = w.layers, w.heads, pipe.S
+    half = w.n_seeds // 2
+    ma = torch.zeros((L, H, S, S), dtype=torch.float32, device=pipe.dev)
+    mb = torch.zeros_like(ma)
+    t0 = time.perf_counter()
+    for l in range(L):
+        vark.vark_scas_accumulate(pipe.cq[l][:half], pipe.ck[l][:half], pipe.cv[l][:half], pipe.sides, pipe.tau[l],
+                                  pipe.bias[l], ma[l], None, pipe.status)
+        vark.vark_scas_accumulate(pipe.cq[l][half:], pipe.ck[l][half:], pipe.cv[l][half:], pipe.sides, pipe.tau[l],
+                                  pipe.bias[l], mb[l], None, pipe.status)
+    torch.cuda.synchronize()
+    assert int(pipe.status.item()) == 0
+    sa = vark.vark_scas_finalize(ma.cpu().numpy())
+    sb = vark.vark_scas_finalize(mb.cpu().numpy())
+    sp, jc = vark.vark_rank_stability(sa, sb, pipe.sides, w.budget_bp, w.n_sinks)
+    return {"seeds": f"{half} vs {w.n_seeds - half} (disjoint)", "spearman": sp, "drop_jaccard": jc,
+            "budget_bp": w.budget_bp, "seconds": time.perf_counter() - t0}
+
+
 def generation_order(pipe, passes, max_over_ranks, sum_over_ranks):
     """The inference flow scale by scale on the same workload and schedule:
     for each scale k, pruned attention of scale k's queries in every layer over
@@ -471,6 +496,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--gen-passes", type=int, default=2)
+    ap.add_argument("--stability", type=int, default=1)
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -603,6 +629,9 @@ def main():
                "d2h_bytes_per_step": d2h, "steps": ke}
         del host_in, host_out
 
+    # ------------------------------------------------ ranking stability (two disjoint seed halves)
+    stab = ranking_stability(pipe) if args.stability else None
+
     # ------------------------------------------------ generation order (scale by scale)
     gen = None
     if args.gen_passes > 0:
@@ -637,7 +666,8 @@ def main():
                        "value_def": "(calibration + pruned attention FLOPs) / step time; step = calibration, "
                                     "S-CAS, schedule, offsets, compaction, pruned attention of all layers"},
             "pruned_attention_tflops": pruned_tflops, "query_tokens_per_s": qtok_s, "compaction_gbs": comp_gbs,
-            "roofline": roof, "kernels": kernels, "generation_order": gen, "cpu_baseline": cpu, "e2e": e2e,
+            "roofline": roof, "kernels": kernels, "generation_order": gen, "ranking_stability": stab,
+            "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches,
             "clocks": clk, "peaks": peaks,
         }

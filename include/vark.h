@@ -269,6 +269,23 @@ int vark_pruned_attention_step(const uint16_t* q, const uint16_t* kc, const uint
 int vark_cache_size_after_layer(const uint8_t* keep, int L, int H, int S, const int32_t* sides, int B, int D,
                                 int64_t* bytes);
 
+/*
+ * vark_rank_stability -- host.  [HeatKV] Results (S-CAS rankings remain stable
+ * with a small calibration set); [Review] Figure 6 caption (stability of S-CAS
+ * head-scale rankings across calibration runs).  Compares the S-CAS of two
+ * calibration runs on disjoint seed sets over the candidate pairs
+ * (l, h, s >= n_sinks):
+ *   spearman      Pearson correlation of the two vectors of average ranks
+ *                 (ties share the mean of their positions); 0 if either is
+ *                 constant;
+ *   drop_jaccard  |D_a & D_b| / |D_a | D_b| of the pairs each run's
+ *                 vark_build_schedule drops at budget_bp (1 if neither drops).
+ *   scas_a, scas_b  host fp64 [L][H][S], finite.
+ * Errors: VARK_E_ARG, VARK_E_SHAPE (n_sinks >= S), VARK_E_BUDGET.
+ */
+int vark_rank_stability(const double* scas_a, const double* scas_b, int L, int H, int S, const int32_t* sides,
+                        uint32_t budget_bp, int n_sinks, double* spearman, double* drop_jaccard);
+
 #ifdef __cplusplus
 }
 #endif

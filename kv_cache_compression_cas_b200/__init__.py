@@ -51,6 +51,7 @@ _SIGNATURES = {
                                         _P, _P, _P]),
     "vark_append_scale": (_I, [_P, _P, _I64, _I, _I, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P, _P, _P]),
     "vark_cache_size_after_layer": (_I, [_P, _I, _I, _I, _P, _I, _I, _P]),
+    "vark_rank_stability": (_I, [_P, _P, _I, _I, _I, _P, _U32, _I, _P, _P]),
 }
 
 
@@ -251,3 +252,16 @@ def vark_cache_size_after_layer(keep: np.ndarray, sides, B: int, D: int) -> np.n
     _check(_load().vark_cache_size_after_layer(kp.ctypes.data, L, H, S, s_ptr, int(B), int(D), out.ctypes.data),
            "vark_cache_size_after_layer")
     return out
+
+
+def vark_rank_stability(scas_a: np.ndarray, scas_b: np.ndarray, sides, budget_bp: int, n_sinks: int):
+    """Host: (spearman, drop_jaccard) of two S-CAS arrays [L][H][S]."""
+    a = np.ascontiguousarray(scas_a, dtype=np.float64)
+    b = np.ascontiguousarray(scas_b, dtype=np.float64)
+    L, H, S = a.shape
+    s_arr, s_ptr = _sides_arg(sides)
+    sp = ctypes.c_double()
+    jc = ctypes.c_double()
+    _check(_load().vark_rank_stability(a.ctypes.data, b.ctypes.data, L, H, S, s_ptr, int(budget_bp), int(n_sinks),
+                                       ctypes.byref(sp), ctypes.byref(jc)), "vark_rank_stability")
+    return sp.value, jc.value

@@ -130,3 +130,63 @@ extern "C" int vark_cache_size_after_layer(const uint8_t* keep, int L, int H, in
   }
   return VARK_OK;
 }
+
+// Average ranks (1-based) of v, ties sharing the mean of their positions.
+static void average_ranks(const std::vector<double>& v, std::vector<double>& rank) {
+  const size_t n = v.size();
+  std::vector<size_t> idx(n);
+  for (size_t i = 0; i < n; ++i) idx[i] = i;
+  std::stable_sort(idx.begin(), idx.end(), [&](size_t a, size_t b) { return v[a] < v[b]; });
+  rank.assign(n, 0.0);
+  for (size_t i = 0; i < n;) {
+    size_t j = i;
+    while (j + 1 < n && v[idx[j + 1]] == v[idx[i]]) ++j;
+    const double r = 0.5 * double(i + j) + 1.0;
+    for (size_t t = i; t <= j; ++t) rank[idx[t]] = r;
+    i = j + 1;
+  }
+}
+
+extern "C" int vark_rank_stability(const double* scas_a, const double* scas_b, int L, int H, int S,
+                                   const int32_t* sides, uint32_t budget_bp, int n_sinks, double* spearman,
+                                   double* drop_jaccard) {
+  if (!scas_a || !scas_b || !sides || !spearman || !drop_jaccard) return VARK_E_ARG;
+  int64_t T = 0;
+  if (L < 1 || H < 1 || !sides_ok(S, sides, &T) || n_sinks < 0 || n_sinks >= S) return VARK_E_SHAPE;
+  std::vector<double> a, b;
+  for (int l = 0; l < L; ++l)
+    for (int h = 0; h < H; ++h)
+      for (int s = n_sinks; s < S; ++s) {
+        const int64_t i = (int64_t(l) * H + h) * S + s;
+        if (!std::isfinite(scas_a[i]) || !std::isfinite(scas_b[i])) return VARK_E_ARG;
+        a.push_back(scas_a[i]);
+        b.push_back(scas_b[i]);
+      }
+  std::vector<double> ra, rb;
+  average_ranks(a, ra);
+  average_ranks(b, rb);
+  const double n = double(ra.size());
+  double ma = 0, mb = 0;
+  for (size_t i = 0; i < ra.size(); ++i) { ma += ra[i]; mb += rb[i]; }
+  ma /= n; mb /= n;
+  double sab = 0, saa = 0, sbb = 0;
+  for (size_t i = 0; i < ra.size(); ++i) {
+    sab += (ra[i] - ma) * (rb[i] - mb);
+    saa += (ra[i] - ma) * (ra[i] - ma);
+    sbb += (rb[i] - mb) * (rb[i] - mb);
+  }
+  *spearman = (saa > 0 && sbb > 0) ? sab / std::sqrt(saa * sbb) : 0.0;
+  std::vector<uint8_t> ka(size_t(int64_t(L) * H * S)), kb(ka.size());
+  int rc = vark_build_schedule(scas_a, L, H, S, sides, budget_bp, n_sinks, ka.data());
+  if (rc) return rc;
+  rc = vark_build_schedule(scas_b, L, H, S, sides, budget_bp, n_sinks, kb.data());
+  if (rc) return rc;
+  int64_t inter = 0, uni = 0;
+  for (size_t i = 0; i < ka.size(); ++i) {
+    const bool da = ka[i] == 0, db = kb[i] == 0;
+    inter += (da && db) ? 1 : 0;
+    uni += (da || db) ? 1 : 0;
+  }
+  *drop_jaccard = uni > 0 ? double(inter) / double(uni) : 1.0;
+  return VARK_OK;
+}

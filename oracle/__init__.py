@@ -33,9 +33,11 @@ from .attention import (block_causal_attention, attend, scas_mass, pruned_attent
 from .schedule import scas_from_mass, build_schedule, BudgetError, full_cache_tokens
 from .layout import build_offsets, compact_kv
 from .generation import append_scale, cache_size_after_layer
+from .stability import rank_stability, average_ranks
 
 __all__ = [
     "ScaleGeometry", "block_causal_attention", "attend", "scas_mass", "pruned_attention",
     "attention_rows", "pruned_attention_rows", "scas_from_mass", "build_schedule", "BudgetError", "full_cache_tokens",
     "build_offsets", "compact_kv", "append_scale", "cache_size_after_layer",
+    "rank_stability", "average_ranks",
 ]

@@ -100,3 +100,18 @@ def test_cache_size_accounting_matches_oracle(sides, L, H):
     keep = np.random.default_rng(L + H).integers(0, 2, size=(L, H, len(sides))).astype(np.uint8)
     got = vark.vark_cache_size_after_layer(keep, sides, 4, 128)
     assert np.array_equal(got, oracle.cache_size_after_layer(keep, sides, 4, 128))
+
+
+def test_rank_stability_matches_oracle():
+    rng = np.random.default_rng(5)
+    for sides, L, H in ((SIDES_TINY, 2, 3), (SIDES_1024, 32, 16)):
+        S = len(sides)
+        a = rng.uniform(size=(L, H, S))
+        b = np.round(a + 0.05 * rng.standard_normal(size=a.shape), 2)
+        for budget in (5000, 1000):
+            try:
+                ref = oracle.rank_stability(a, b, sides, budget, 2)
+            except oracle.BudgetError:
+                continue
+            got = vark.vark_rank_stability(a, b, sides, budget, 2)
+            assert abs(got[0] - ref[0]) < 1e-12 and got[1] == ref[1]

@@ -441,3 +441,22 @@ def test_cache_size_accounting_closed_forms():
     assert np.all(np.diff(sz.ravel()) >= 0)
     _, _, _, lb = oracle.build_offsets(keep, sides, B, D)
     assert sz[-1, -1] == 4 * int(lb[-1])
+
+
+# ---------------------------------------------------------------- ranking stability
+
+def test_rank_stability_pins():
+    from scipy.stats import spearmanr
+    sides = SIDES_TINY
+    rng = np.random.default_rng(21)
+    a = rng.uniform(size=(2, 3, 7))
+    b = a + 0.1 * rng.standard_normal(size=a.shape)
+    b[0, 0, 2:4] = b[0, 0, 5]                     # ties
+    sp, jc = oracle.rank_stability(a, b, sides, 5000, 2)
+    ref = spearmanr(a[:, :, 2:].ravel(), b[:, :, 2:].ravel()).correlation
+    assert abs(sp - ref) < 1e-12
+    sp1, jc1 = oracle.rank_stability(a, a, sides, 5000, 2)
+    assert abs(sp1 - 1.0) < 1e-12 and jc1 == 1.0
+    sp2, _ = oracle.rank_stability(a, -a, sides, 5000, 2)
+    assert abs(sp2 + 1.0) < 1e-12
+    assert 0.0 <= jc <= 1.0
