@@ -286,6 +286,47 @@ int vark_cache_size_after_layer(const uint8_t* keep, int L, int H, int S, const 
 int vark_rank_stability(const double* scas_a, const double* scas_b, int L, int H, int S, const int32_t* sides,
                         uint32_t budget_bp, int n_sinks, double* spearman, double* drop_jaccard);
 
+/* ---------------------------------------------------------------------------
+ * Time-varying schedule: BINARY-HEATKV with GREEDYEARLYPRUNING.  [Review]
+ * Figure 4 caption (Algorithm 1): per source scale i an order O_i ranks the
+ * (layer, head) squares from least to most dependent on scale i; after scale k,
+ * G_k = union over i <= k of the length-N_k prefixes of O_i must be absent.
+ * [HeatKV] Method step 5: cache use stays within the budget as scales are
+ * generated.  The pages leave N_k undefined; this library's reading: the
+ * budget is absolute (budget_bp / 10000 of the final full cache) and N_k is
+ * the smallest non-decreasing prefix length under which the cache after step k
+ * (sink scales of every head, non-sink scales <= k of the heads outside the
+ * prefixes) fits it.  Cache held after step k:
+ *     keep_k[l][h][i] = (i <= k) and (evict_step[l][h][i] > k).
+ * ------------------------------------------------------------------------- */
+
+/*
+ * vark_build_early_pruning_schedule -- host.
+ *   scas        host fp64 [L][H][S]; O_i = ascending (scas[l][h][i], l, h).
+ *   prefix_len  host int32 [S] out: N_k (0 while no non-sink scale exists).
+ *   evict_step  host uint8 [L][H][S] out: first step k >= i at which (l, h, i)
+ *               must be absent, 255 if it stays to the end (always 255 for
+ *               sink scales).  S <= 254.
+ * Errors: VARK_E_ARG, VARK_E_SHAPE, VARK_E_BUDGET (sinks alone over budget).
+ */
+int vark_build_early_pruning_schedule(const double* scas, int L, int H, int S, const int32_t* sides,
+                                      uint32_t budget_bp, int n_sinks, int32_t* prefix_len, uint8_t* evict_step);
+
+/*
+ * vark_recompact_kv -- device.  Moves a compacted cache to the layout of a
+ * smaller (or shifted) retained set, e.g. keep_k after evictions: for every
+ * (l, b, h, s) with keep_new[l][h][s] and s < max_scale, copies the rows from
+ * the old layout (old tables) to the new one (tables of vark_build_offsets on
+ * keep_new).  Pairs absent from the old layout (seg_off_old < 0) are skipped.
+ * Source and destination buffers must differ.
+ * Errors: VARK_E_ARG, VARK_E_SHAPE, VARK_E_ALIGN, VARK_E_CUDA.
+ */
+int vark_recompact_kv(const uint16_t* kc_old, const uint16_t* vc_old, const int32_t* head_off_old,
+                      const int32_t* seg_off_old, const int64_t* layer_base_old,
+                      int L, int B, int H, int S, int D, const int32_t* sides, int max_scale,
+                      const uint8_t* keep_new, const int32_t* head_off_new, const int32_t* seg_off_new,
+                      const int64_t* layer_base_new, uint16_t* kc_new, uint16_t* vc_new, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

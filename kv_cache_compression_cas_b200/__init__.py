@@ -52,6 +52,8 @@ _SIGNATURES = {
     "vark_append_scale": (_I, [_P, _P, _I64, _I, _I, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P, _P, _P]),
     "vark_cache_size_after_layer": (_I, [_P, _I, _I, _I, _P, _I, _I, _P]),
     "vark_rank_stability": (_I, [_P, _P, _I, _I, _I, _P, _U32, _I, _P, _P]),
+    "vark_build_early_pruning_schedule": (_I, [_P, _I, _I, _I, _P, _U32, _I, _P, _P]),
+    "vark_recompact_kv": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P, _P, _P]),
 }
 
 
@@ -265,3 +267,32 @@ def vark_rank_stability(scas_a: np.ndarray, scas_b: np.ndarray, sides, budget_bp
     _check(_load().vark_rank_stability(a.ctypes.data, b.ctypes.data, L, H, S, s_ptr, int(budget_bp), int(n_sinks),
                                        ctypes.byref(sp), ctypes.byref(jc)), "vark_rank_stability")
     return sp.value, jc.value
+
+
+def vark_build_early_pruning_schedule(scas: np.ndarray, sides, budget_bp: int, n_sinks: int):
+    """Host: (prefix_len int32 [S], evict_step uint8 [L][H][S])."""
+    sc = np.ascontiguousarray(scas, dtype=np.float64)
+    L, H, S = sc.shape
+    s_arr, s_ptr = _sides_arg(sides)
+    prefix = np.zeros(S, dtype=np.int32)
+    evict = np.zeros((L, H, S), dtype=np.uint8)
+    _check(_load().vark_build_early_pruning_schedule(sc.ctypes.data, L, H, S, s_ptr, int(budget_bp), int(n_sinks),
+                                                     prefix.ctypes.data, evict.ctypes.data),
+           "vark_build_early_pruning_schedule")
+    return prefix, evict
+
+
+def vark_recompact_kv(kc_old, vc_old, head_off_old, seg_off_old, layer_base_old, L: int, B: int, H: int, sides,
+                      D: int, max_scale: int, keep_new, head_off_new, seg_off_new, layer_base_new, kc_new, vc_new,
+                      stream=None):
+    """Device: move a compacted cache into the layout of a new retained set."""
+    import torch
+    s_arr, s_ptr = _sides_arg(sides)
+    rc = _load().vark_recompact_kv(
+        _dptr(kc_old, torch.bfloat16, "kc_old"), _dptr(vc_old, torch.bfloat16, "vc_old"),
+        _dptr(head_off_old, torch.int32, "head_off_old"), _dptr(seg_off_old, torch.int32, "seg_off_old"),
+        _dptr(layer_base_old, torch.int64, "layer_base_old"), int(L), int(B), int(H), len(s_arr), int(D), s_ptr,
+        int(max_scale), _dptr(keep_new, torch.uint8, "keep_new"), _dptr(head_off_new, torch.int32, "head_off_new"),
+        _dptr(seg_off_new, torch.int32, "seg_off_new"), _dptr(layer_base_new, torch.int64, "layer_base_new"),
+        _dptr(kc_new, torch.bfloat16, "kc_new"), _dptr(vc_new, torch.bfloat16, "vc_new"), _stream(stream))
+    _check(rc, "vark_recompact_kv")

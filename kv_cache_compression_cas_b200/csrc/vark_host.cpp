@@ -190,3 +190,58 @@ extern "C" int vark_rank_stability(const double* scas_a, const double* scas_b, i
   *drop_jaccard = uni > 0 ? double(inter) / double(uni) : 1.0;
   return VARK_OK;
 }
+
+extern "C" int vark_build_early_pruning_schedule(const double* scas, int L, int H, int S, const int32_t* sides,
+                                                 uint32_t budget_bp, int n_sinks, int32_t* prefix_len,
+                                                 uint8_t* evict_step) {
+  if (scas == nullptr || sides == nullptr || prefix_len == nullptr || evict_step == nullptr) return VARK_E_ARG;
+  if (budget_bp > 10000u || n_sinks < 0) return VARK_E_ARG;
+  int64_t T = 0;
+  if (L < 1 || H < 1 || !sides_ok(S, sides, &T) || n_sinks > S || S > 254) return VARK_E_SHAPE;
+  const int64_t LH = int64_t(L) * H;
+  const int64_t LHS = LH * S;
+  for (int64_t i = 0; i < LHS; ++i)
+    if (!std::isfinite(scas[i])) return VARK_E_ARG;
+  // Absolute budget in tokens: budget_bp / 10000 of the final full cache.
+  const int64_t F = LH * T;
+  const int64_t budget = int64_t(budget_bp);
+  int64_t sink_tokens = 0;
+  for (int s = 0; s < n_sinks; ++s) sink_tokens += LH * int64_t(sides[s]) * sides[s];
+  if (sink_tokens * 10000 > budget * F) return VARK_E_BUDGET;
+  // rank[i][(l, h)] = position of (l, h) in O_i: ascending (scas[l][h][i], l, h)
+  std::vector<int64_t> rank(size_t(LH) * S, 0);
+  std::vector<int64_t> order(static_cast<size_t>(LH));
+  for (int i = n_sinks; i < S; ++i) {
+    for (int64_t lh = 0; lh < LH; ++lh) order[size_t(lh)] = lh;
+    std::sort(order.begin(), order.end(), [&](int64_t a, int64_t b) {
+      const double va = scas[a * S + i], vb = scas[b * S + i];
+      if (va != vb) return va < vb;
+      return a < b;
+    });
+    for (int64_t pos = 0; pos < LH; ++pos) rank[size_t(i) * LH + order[size_t(pos)]] = pos;
+  }
+  // N_k: smallest prefix length (non-decreasing in k) whose retained cache
+  // after step k, sinks + (LH - N_k) heads of every non-sink scale <= k, fits.
+  int64_t N = 0;
+  for (int k = 0; k < S; ++k) {
+    int64_t nonsink = 0;
+    for (int i = n_sinks; i <= k; ++i) nonsink += int64_t(sides[i]) * sides[i];
+    int64_t sinks_k = 0;
+    for (int i = 0; i < n_sinks && i <= k; ++i) sinks_k += LH * int64_t(sides[i]) * sides[i];
+    while (N < LH && (sinks_k + (LH - N) * nonsink) * 10000 > budget * F) ++N;
+    prefix_len[k] = int32_t(nonsink > 0 ? N : 0);
+  }
+  // evict_step[l][h][i]: first step k >= i with rank_i(l, h) < N_k; 255 = kept to the end
+  for (int64_t lh = 0; lh < LH; ++lh)
+    for (int i = 0; i < S; ++i) {
+      uint8_t e = 255;
+      if (i >= n_sinks)
+        for (int k = i; k < S; ++k)
+          if (rank[size_t(i) * LH + lh] < prefix_len[k]) {
+            e = uint8_t(k);
+            break;
+          }
+      evict_step[lh * S + i] = e;
+    }
+  return VARK_OK;
+}

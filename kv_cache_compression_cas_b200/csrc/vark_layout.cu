@@ -79,6 +79,10 @@ struct CompactParams {
   int l0, nl;                       // layer group [l0, l0 + nl)
   int L, B, H, D;
   int64_t layer_stride;             // elements between source layers
+  // compacted source (re-compaction): the source's own offset tables
+  const int32_t* src_head_off;      // null: dense source
+  const int32_t* src_seg_off;
+  const int64_t* src_layer_base;
 };
 
 __global__ void __launch_bounds__(kCompactThreads) compact_kernel(
@@ -169,9 +173,18 @@ __global__ void __launch_bounds__(kCompactThreads) compact_kernel(
     const int32_t nrows = min(kChunkRows, p.sc.n[s] - r0);
     const int64_t R_l = (layer_base[l + 1] - layer_base[l]) / (int64_t(p.B) * p.D);
     const int64_t dst_row = int64_t(b) * R_l + head_off[l * H + h] + seg_off[(l * H + h) * S + s] + r0;
-    const int64_t src_row = (int64_t(b) * H + h) * p.src_rows + p.src_off[s] + r0;
     const int64_t dst_v = (layer_base[l] / 8) + dst_row * vec_per_row;
-    const int64_t src_v = (int64_t(l) * p.layer_stride) / 8 + src_row * vec_per_row;
+    int64_t src_v;
+    if (p.src_head_off == nullptr) {
+      const int64_t src_row = (int64_t(b) * H + h) * p.src_rows + p.src_off[s] + r0;
+      src_v = (int64_t(l) * p.layer_stride) / 8 + src_row * vec_per_row;
+    } else {
+      const int32_t so = p.src_seg_off[(l * H + h) * S + s];
+      if (so < 0) continue;   // not in the source: nothing to move
+      const int64_t R_src = (p.src_layer_base[l + 1] - p.src_layer_base[l]) / (int64_t(p.B) * p.D);
+      const int64_t src_row = int64_t(b) * R_src + p.src_head_off[l * H + h] + so + r0;
+      src_v = p.src_layer_base[l] / 8 + src_row * vec_per_row;
+    }
     const int nvec = nrows * vec_per_row;
 
     // 4 K + 4 V vectors in flight per thread, then the stores.
@@ -223,9 +236,11 @@ extern "C" int vark_build_offsets(const uint8_t* keep, int L, int H, int S, cons
 // as [B][H][src_rows][D] with scale s starting at row src_off[s].
 static int launch_gather(const uint16_t* k, const uint16_t* v, int64_t layer_stride, int L, int B, int H, int D,
                          CompactParams& p, int s_lo, int s_hi, int64_t src_rows, const int32_t* src_off,
+                         const int32_t* src_head_off, const int32_t* src_seg_off, const int64_t* src_layer_base,
                          const uint8_t* keep, const int32_t* head_off, const int32_t* seg_off,
                          const int64_t* layer_base, uint16_t* kc, uint16_t* vc, cudaStream_t st) {
   p.L = L; p.B = B; p.H = H; p.D = D; p.layer_stride = layer_stride; p.src_rows = src_rows;
+  p.src_head_off = src_head_off; p.src_seg_off = src_seg_off; p.src_layer_base = src_layer_base;
   for (int s = 0; s < VARK_MAX_SCALES; ++s) {
     const bool in = s < p.sc.S && s >= s_lo && s < s_hi;
     p.chunks[s] = in ? (p.sc.n[s] + kChunkRows - 1) / kChunkRows : 0;
@@ -261,8 +276,8 @@ extern "C" int vark_compact_kv(const uint16_t* k, const uint16_t* v, int64_t lay
   if (layer_stride % 8 != 0) return VARK_E_ALIGN;
   if (!aligned16(k) || !aligned16(v) || !aligned16(kc) || !aligned16(vc)) return VARK_E_ALIGN;
   if ((rc = check_device_sm100())) return rc;
-  return launch_gather(k, v, layer_stride, L, B, H, D, p, 0, S, p.sc.T, p.sc.off, keep, head_off, seg_off,
-                       layer_base, kc, vc, static_cast<cudaStream_t>(stream));
+  return launch_gather(k, v, layer_stride, L, B, H, D, p, 0, S, p.sc.T, p.sc.off, nullptr, nullptr, nullptr, keep,
+                       head_off, seg_off, layer_base, kc, vc, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" int vark_append_scale(const uint16_t* k_new, const uint16_t* v_new, int64_t layer_stride, int L, int B,
@@ -281,6 +296,31 @@ extern "C" int vark_append_scale(const uint16_t* k_new, const uint16_t* v_new, i
   if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(kc) || !aligned16(vc)) return VARK_E_ALIGN;
   if ((rc = check_device_sm100())) return rc;
   int32_t zero_off[VARK_MAX_SCALES] = {0};
-  return launch_gather(k_new, v_new, layer_stride, L, B, H, D, p, scale, scale + 1, p.sc.n[scale], zero_off, keep,
-                       head_off, seg_off, layer_base, kc, vc, static_cast<cudaStream_t>(stream));
+  return launch_gather(k_new, v_new, layer_stride, L, B, H, D, p, scale, scale + 1, p.sc.n[scale], zero_off, nullptr,
+                       nullptr, nullptr, keep, head_off, seg_off, layer_base, kc, vc,
+                       static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int vark_recompact_kv(const uint16_t* kc_old, const uint16_t* vc_old, const int32_t* head_off_old,
+                                 const int32_t* seg_off_old, const int64_t* layer_base_old, int L, int B, int H,
+                                 int S, int D, const int32_t* sides, int max_scale, const uint8_t* keep_new,
+                                 const int32_t* head_off_new, const int32_t* seg_off_new,
+                                 const int64_t* layer_base_new, uint16_t* kc_new, uint16_t* vc_new, void* stream) {
+  if (!kc_old || !vc_old || !head_off_old || !seg_off_old || !layer_base_old || !keep_new || !head_off_new ||
+      !seg_off_new || !layer_base_new || !kc_new || !vc_new)
+    return VARK_E_ARG;
+  if (kc_old == kc_new || vc_old == vc_new) return VARK_E_ARG;
+  CompactParams p;
+  int rc = make_scale_table(S, sides, &p.sc);
+  if (rc) return rc;
+  if (max_scale < 0 || max_scale > S) return VARK_E_ARG;
+  if (L < 1 || H < 1 || B < 1 || D < 8 || D % 8 != 0 || D > 1024) return VARK_E_SHAPE;
+  if (H > kMaxGroupLH) return VARK_E_SHAPE;
+  if (!aligned16(kc_old) || !aligned16(vc_old) || !aligned16(kc_new) || !aligned16(vc_new)) return VARK_E_ALIGN;
+  if ((rc = check_device_sm100())) return rc;
+  if (max_scale == 0) return VARK_OK;
+  int32_t zero_off[VARK_MAX_SCALES] = {0};
+  return launch_gather(kc_old, vc_old, 0, L, B, H, D, p, 0, max_scale, 0, zero_off, head_off_old, seg_off_old,
+                       layer_base_old, keep_new, head_off_new, seg_off_new, layer_base_new, kc_new, vc_new,
+                       static_cast<cudaStream_t>(stream));
 }

@@ -115,3 +115,12 @@ def test_rank_stability_matches_oracle():
                 continue
             got = vark.vark_rank_stability(a, b, sides, budget, 2)
             assert abs(got[0] - ref[0]) < 1e-12 and got[1] == ref[1]
+
+
+@pytest.mark.parametrize("sides,L,H,budget", [(SIDES_TINY, 2, 3, 2500), (SIDES_1024, 32, 16, 1000),
+                                               (SIDES_1024, 8, 32, 400)])
+def test_early_pruning_schedule_matches_oracle(sides, L, H, budget):
+    scas = np.round(np.random.default_rng(L * H).uniform(size=(L, H, len(sides))), 3)
+    p_ref, e_ref = oracle.early_pruning_schedule(scas, sides, budget, 2)
+    p_got, e_got = vark.vark_build_early_pruning_schedule(scas, sides, budget, 2)
+    assert np.array_equal(p_got, p_ref) and np.array_equal(e_got, e_ref)

@@ -460,3 +460,40 @@ def test_rank_stability_pins():
     sp2, _ = oracle.rank_stability(a, -a, sides, 5000, 2)
     assert abs(sp2 + 1.0) < 1e-12
     assert 0.0 <= jc <= 1.0
+
+
+# ---------------------------------------------------------------- time-varying schedule
+
+@pytest.mark.parametrize("budget", [10000, 5000, 2500, 1200])
+def test_early_pruning_schedule_brute_force(budget):
+    """N_k is the smallest non-decreasing prefix length keeping every step's
+    retained cache within the absolute budget; evictions follow the O_i."""
+    sides = SIDES_TINY
+    g = _geom(sides)
+    L, H, n_sinks = 2, 3, 2
+    LH = L * H
+    scas = np.round(np.random.default_rng(budget).uniform(size=(L, H, g.S)), 2)
+    prefix, evict = oracle.early_pruning_schedule(scas, sides, budget, n_sinks)
+    F = LH * g.T
+    prev = 0
+    for k in range(g.S):
+        def retained(N):
+            return sum(LH * g.n[i] for i in range(min(n_sinks, k + 1))) + \
+                sum((LH - N) * g.n[i] for i in range(n_sinks, k + 1))
+        feasible = [N for N in range(prev, LH + 1) if retained(N) * 10000 <= budget * F]
+        want = feasible[0] if feasible else LH
+        if k < n_sinks:
+            want = 0
+        assert prefix[k] == want, (k, prefix[k], want)
+        prev = max(prev, prefix[k])
+        keep_k = oracle.keep_after_step(evict, k)
+        held = int((keep_k * np.array(g.n)[None, None, :]).sum())
+        if feasible:
+            assert held * 10000 <= budget * F
+        # evicted pairs of scale i are exactly the N_k least dependent (l, h) on i
+        for i in range(n_sinks, k + 1):
+            gone = {lh for lh in range(LH) if not keep_k.reshape(LH, g.S)[lh, i]}
+            order = sorted(range(LH), key=lambda lh: (scas.reshape(LH, g.S)[lh, i], lh))
+            assert gone == set(order[:prefix[k]])
+    if budget == 10000:
+        assert np.all(evict == 255)
