@@ -217,6 +217,7 @@ class Pipeline:
         st.synchronize()
         scas = vark.vark_scas_finalize(self.mass_host.numpy())
         keep = vark.vark_build_schedule(scas, self.sides, w.budget_bp, w.n_sinks)
+        self.last_scas = scas
         self.keep_host.numpy()[...] = keep
         self.keep.copy_(self.keep_host, non_blocking=True)
         rec("sched")
@@ -477,12 +478,98 @@ def generation_order(pipe, passes, max_over_ranks, sum_over_ranks):
     nl = np.array(n, dtype=np.int64)
     kept_rows = int((keep.astype(np.int64) * nl[None, None, :]).sum())
     app_bytes = 2.0 * kept_rows * B * D * 2 * 2 * passes
+    static = {"passes": passes, "ms_per_pass": t * 1e3 / passes,
+              "attention_tflops": sum_over_ranks(fl) / attn_s / 1e12,
+              "append_and_zero_ms_per_pass": (t - attn_s) * 1e3 / passes,
+              "query_tokens_per_s": sum_over_ranks(float(L * B * pipe.T * passes)) / t,
+              "append_bytes_per_pass": app_bytes / passes,
+              "peak_cache_bytes": 4 * int(base[-1]),
+              "launches_per_pass": len(sides) * (L + 1) + 2}
+    return {"static_schedule": static,
+            "early_pruning": early_pruning_order(pipe, per_scale, outs, passes, max_over_ranks, sum_over_ranks)}
+
+
+def early_pruning_order(pipe, per_scale, outs, passes, max_over_ranks, sum_over_ranks):
+    """Scale by scale under the time-varying schedule (BINARY-HEATKV with
+    GREEDYEARLYPRUNING, the library's reading) at the same absolute budget:
+    attention over the cache held after the previous step, then the survivors
+    move to the new layout and the new scale is appended."""
+    import torch
+    vark, w = pipe.vark, pipe.w
+    L, B, H, D, S = w.layers, w.batch, w.heads, w.head_dim, pipe.S
+    sides = pipe.sides
+    n = np.array([s * s for s in sides], dtype=np.int64)
+    prefix, evict = vark.vark_build_early_pruning_schedule(pipe.last_scas, sides, w.budget_bp, w.n_sinks)
+    idx = np.arange(S)[None, None, :]
+    keeps = [((idx <= k) & (evict.astype(np.int64) > k)).astype(np.uint8) for k in range(S)]
+    held = [int((kp * n[None, None, :]).sum()) for kp in keeps]
+    cap = B * D * (max(held) + int(n.max()) + 1)
+    dev = pipe.dev
+    bufs = [(torch.zeros(cap, dtype=torch.bfloat16, device=dev), torch.zeros(cap, dtype=torch.bfloat16, device=dev))
+            for _ in range(2)]
+    tabs = []
+    for k in range(S):                               # tables of every step's retained set (schedule data)
+        kp = torch.from_numpy(keeps[k]).to(dev)
+        t = {"keep": kp, "head_off": torch.empty((L, H), dtype=torch.int32, device=dev),
+             "seg_off": torch.empty((L, H, S), dtype=torch.int32, device=dev),
+             "past_len": torch.empty((L, H, S), dtype=torch.int32, device=dev),
+             "layer_base": torch.empty(L + 1, dtype=torch.int64, device=dev)}
+        vark.vark_build_offsets(kp, sides, B, D, t["head_off"], t["seg_off"], t["past_len"], t["layer_base"])
+        t["base"] = t["layer_base"].cpu().numpy()
+        tabs.append(t)
+    empty = {"keep": torch.zeros((L, H, S), dtype=torch.uint8, device=dev)}
+    for key in ("head_off",):
+        empty[key] = torch.zeros((L, H), dtype=torch.int32, device=dev)
+    empty["seg_off"] = torch.full((L, H, S), -1, dtype=torch.int32, device=dev)
+    empty["past_len"] = torch.zeros((L, H, S), dtype=torch.int32, device=dev)
+    empty["layer_base"] = torch.zeros(L + 1, dtype=torch.int64, device=dev)
+    empty["base"] = np.zeros(L + 1, dtype=np.int64)
+    st = torch.cuda.current_stream()
+    moved = 0
+
+    def one_pass():
+        nonlocal moved
+        moved = 0
+        prev, (kcp, vcp) = empty, bufs[1]
+        for k, (qk, kk, vk) in enumerate(per_scale):
+            for l in range(L):
+                rows = int(prev["base"][l + 1] - prev["base"][l]) // D
+                b0, b1 = int(prev["base"][l]), int(prev["base"][l + 1])
+                vark.vark_pruned_attention_step(qk[l], kcp[b0:b1] if rows else None, vcp[b0:b1] if rows else None,
+                                                rows, kk[l], vk[l], sides, k, prev["head_off"][l],
+                                                prev["seg_off"][l], prev["past_len"][l], pipe.tau[l], pipe.bias[l],
+                                                outs[k][l], pipe.status)
+            t = tabs[k]
+            kcn, vcn = bufs[k % 2]
+            vark.vark_recompact_kv(kcp, vcp, prev["head_off"], prev["seg_off"], prev["layer_base"], L, B, H, sides,
+                                   D, k, t["keep"], t["head_off"], t["seg_off"], t["layer_base"], kcn, vcn)
+            vark.vark_append_scale(kk, vk, B * H * int(n[k]) * D, L, B, H, sides, D, k, t["keep"], t["head_off"],
+                                   t["seg_off"], t["layer_base"], kcn, vcn)
+            moved += 2 * 2 * 2 * int(t["base"][-1])   # read + write, K and V, bf16 (survivors + appended rows)
+            prev, (kcp, vcp) = t, (kcn, vcn)
+
+    one_pass()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(passes):
+        one_pass()
+    e1.record(st)
+    torch.cuda.synchronize()
+    assert int(pipe.status.item()) == 0
+    t = max_over_ranks(e0.elapsed_time(e1) / 1e3)
+    nl = n.astype(np.float64)
+    fl = 0.0
+    for k in range(S):
+        kp = keeps[k - 1] if k > 0 else np.zeros_like(keeps[0])
+        past = (kp[:, :, :k].astype(np.float64) * nl[None, None, :k]).sum(axis=2)
+        fl += float((4.0 * B * nl[k] * (past + nl[k]) * D).sum())
     return {"passes": passes, "ms_per_pass": t * 1e3 / passes,
-            "attention_tflops": sum_over_ranks(fl) / attn_s / 1e12,
-            "append_and_zero_ms_per_pass": (t - attn_s) * 1e3 / passes,
+            "attention_tflops_incl_moves": sum_over_ranks(fl * passes) / t / 1e12,
             "query_tokens_per_s": sum_over_ranks(float(L * B * pipe.T * passes)) / t,
-            "append_bytes_per_pass": app_bytes / passes,
-            "launches_per_pass": len(sides) * (L + 1) + 2}
+            "prefix_len": [int(x) for x in prefix],
+            "peak_cache_bytes": 4 * B * D * max(held), "final_cache_bytes": 4 * B * D * held[-1],
+            "bytes_moved_per_pass": moved}
 
 
 def reduce_over_ranks(x: float, op: str, world: int, device) -> float:
