@@ -49,6 +49,11 @@ constexpr int kStages = 2;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxPairs = 512;
 constexpr int kMaxDesc = 256;            // key tiles with a precomputed descriptor
+// (batch, head) blocks interleaved in the launch order: pruned attention
+// gains from ending each launch on light CTAs; calibration, whose per-head
+// K/V is larger, measured best head by head.
+template <bool PRUNED>
+struct HeadGroup { static constexpr int value = PRUNED ? 8 : 1; };
 constexpr int kPanelBytes = 128 * 128;   // 128 rows x 128 bytes (64 bf16)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 domain
@@ -159,9 +164,19 @@ struct Item {
 template <bool PRUNED>
 __device__ Item<PRUNED> decode_item(const Params& p) {
   Item<PRUNED> it;
-  // (batch, head)-major order: the CTAs in flight share a few heads' K/V in L2.
-  it.bh = blockIdx.x / p.n_pairs;
-  const int pi = blockIdx.x % p.n_pairs;
+  // Groups of G (batch, head) blocks, one after another: the CTAs in
+  // flight share a few heads' K/V in L2.  Inside a group the order is pair-
+  // major (heaviest pair of every head of the group first), so each launch
+  // ends on light CTAs instead of a last head's heaviest ones.
+  const int BH = p.B * p.H;
+  constexpr int G = HeadGroup<PRUNED>::value;
+  const int per_group = G * p.n_pairs;
+  const int grp = blockIdx.x / per_group;
+  const int g0 = grp * G;
+  const int gsize = min(G, BH - g0);
+  const int within = blockIdx.x - grp * per_group;
+  it.bh = g0 + within % gsize;
+  const int pi = within / gsize;
   it.b = it.bh / p.H;
   it.h = it.bh % p.H;
   const uint32_t e = p.pair[pi];
