@@ -327,6 +327,46 @@ int vark_recompact_kv(const uint16_t* kc_old, const uint16_t* vc_old, const int3
                       const uint8_t* keep_new, const int32_t* head_off_new, const int32_t* seg_off_new,
                       const int64_t* layer_base_new, uint16_t* kc_new, uint16_t* vc_new, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Quantised retained cache (int8).  [VAR-Q] summary page: KV quantisation for
+ * visual AR models with groups indexed by (block, channel), block boundaries
+ * given by the generation loop, composable with eviction.  Here a block is one
+ * retained scale of one (layer, batch, head) and every channel d of it has one
+ * absmax a (fp32); code = rint(x / (a / 127)) clamped to [-127, 127] (IEEE fp32
+ * division, round half to even; a = 0 gives code 0); x' = code * (a / 127),
+ * rounded to bf16.  Codes sit at the element positions of the compacted layout
+ * (one byte each); absmax tables are [L][B][H][S][D] fp32 (entries of dropped
+ * scales are 0).
+ * ------------------------------------------------------------------------- */
+
+/*
+ * vark_quantize_kv_int8 -- device.  Compaction with quantisation: like
+ * vark_compact_kv, but writes int8 codes to kq / vq (layer_base[L] bytes each)
+ * and the per-(block, channel) absmax to k_absmax / v_absmax.  Reads each kept
+ * block twice (absmax pass, code pass).
+ * Errors: VARK_E_ARG, VARK_E_SHAPE (D % 8 != 0, D > 512), VARK_E_ALIGN, VARK_E_CUDA.
+ */
+int vark_quantize_kv_int8(const uint16_t* k, const uint16_t* v, int64_t layer_stride,
+                          int L, int B, int H, int S, int D, const int32_t* sides,
+                          const uint8_t* keep, const int32_t* head_off, const int32_t* seg_off,
+                          const int64_t* layer_base, int8_t* kq, int8_t* vq,
+                          float* k_absmax, float* v_absmax, void* stream);
+
+/*
+ * vark_dequantize_layer_int8 -- device.  Expands one layer's int8 codes back to
+ * its bf16 compacted block (the input of vark_pruned_attention), e.g. into a
+ * one-layer buffer just before that layer's attention.
+ *   kq, vq        dev int8, the layer's codes (kq + layer_base[l]), kc_rows rows.
+ *   k_absmax, v_absmax  dev fp32 [B][H][S][D], the layer's absmax tables.
+ *   head_off, seg_off   dev int32 [H], [H][S]: the layer's offset tables.
+ *   kc, vc        dev bf16 [kc_rows][D] out.
+ * Errors: VARK_E_ARG, VARK_E_SHAPE, VARK_E_ALIGN, VARK_E_CUDA.
+ */
+int vark_dequantize_layer_int8(const int8_t* kq, const int8_t* vq, const float* k_absmax, const float* v_absmax,
+                               int64_t kc_rows, int B, int H, int S, int D, const int32_t* sides,
+                               const int32_t* head_off, const int32_t* seg_off,
+                               uint16_t* kc, uint16_t* vc, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -54,6 +54,8 @@ _SIGNATURES = {
     "vark_rank_stability": (_I, [_P, _P, _I, _I, _I, _P, _U32, _I, _P, _P]),
     "vark_build_early_pruning_schedule": (_I, [_P, _I, _I, _I, _P, _U32, _I, _P, _P]),
     "vark_recompact_kv": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P, _P, _P]),
+    "vark_quantize_kv_int8": (_I, [_P, _P, _I64, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "vark_dequantize_layer_int8": (_I, [_P, _P, _P, _P, _I64, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
 }
 
 
@@ -296,3 +298,30 @@ def vark_recompact_kv(kc_old, vc_old, head_off_old, seg_off_old, layer_base_old,
         _dptr(seg_off_new, torch.int32, "seg_off_new"), _dptr(layer_base_new, torch.int64, "layer_base_new"),
         _dptr(kc_new, torch.bfloat16, "kc_new"), _dptr(vc_new, torch.bfloat16, "vc_new"), _stream(stream))
     _check(rc, "vark_recompact_kv")
+
+
+def vark_quantize_kv_int8(k, v, layer_stride: int, L: int, B: int, H: int, sides, D: int, keep, head_off, seg_off,
+                          layer_base, kq, vq, k_absmax, v_absmax, stream=None):
+    """Device: compaction into int8 codes + per-(block, channel) absmax."""
+    import torch
+    s_arr, s_ptr = _sides_arg(sides)
+    rc = _load().vark_quantize_kv_int8(
+        _dptr(k, torch.bfloat16, "k"), _dptr(v, torch.bfloat16, "v"), int(layer_stride), int(L), int(B), int(H),
+        len(s_arr), int(D), s_ptr, _dptr(keep, torch.uint8, "keep"), _dptr(head_off, torch.int32, "head_off"),
+        _dptr(seg_off, torch.int32, "seg_off"), _dptr(layer_base, torch.int64, "layer_base"),
+        _dptr(kq, torch.int8, "kq"), _dptr(vq, torch.int8, "vq"), _dptr(k_absmax, torch.float32, "k_absmax"),
+        _dptr(v_absmax, torch.float32, "v_absmax"), _stream(stream))
+    _check(rc, "vark_quantize_kv_int8")
+
+
+def vark_dequantize_layer_int8(kq, vq, k_absmax, v_absmax, kc_rows: int, B: int, H: int, sides, D: int, head_off,
+                               seg_off, kc, vc, stream=None):
+    """Device: one layer's int8 codes back to its bf16 compacted block."""
+    import torch
+    s_arr, s_ptr = _sides_arg(sides)
+    rc = _load().vark_dequantize_layer_int8(
+        _dptr(kq, torch.int8, "kq"), _dptr(vq, torch.int8, "vq"), _dptr(k_absmax, torch.float32, "k_absmax"),
+        _dptr(v_absmax, torch.float32, "v_absmax"), int(kc_rows), int(B), int(H), len(s_arr), int(D), s_ptr,
+        _dptr(head_off, torch.int32, "head_off"), _dptr(seg_off, torch.int32, "seg_off"),
+        _dptr(kc, torch.bfloat16, "kc"), _dptr(vc, torch.bfloat16, "vc"), _stream(stream))
+    _check(rc, "vark_dequantize_layer_int8")

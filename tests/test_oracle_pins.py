@@ -497,3 +497,26 @@ def test_early_pruning_schedule_brute_force(budget):
             assert gone == set(order[:prefix[k]])
     if budget == 10000:
         assert np.all(evict == 255)
+
+
+# ---------------------------------------------------------------- int8 retained cache
+
+def test_int8_block_quantisation_pins():
+    from synth import f32_to_bf16_bits
+    rng = np.random.default_rng(4)
+    x = f32_to_bf16_bits(rng.standard_normal((300, 16)).astype(np.float32) * 3)
+    codes, a = oracle.quantize_block(x)
+    back = bf16_bits_to_f32(oracle.dequantize_block(codes, a)).astype(np.float64)
+    xf = bf16_bits_to_f32(x).astype(np.float64)
+    bound = a.astype(np.float64)[None, :] / 254.0 + np.abs(back) * 2.0 ** -8
+    assert np.all(np.abs(back - xf) <= bound + 1e-12)
+    assert np.all(np.abs(codes.astype(np.int64)).max(axis=0) == 127)   # the absmax element maps to +-127
+    # integers in [-127, 127] with absmax 127: scale 1, exact round trip
+    ints = rng.integers(-127, 128, size=(50, 8)).astype(np.float32)
+    ints[0] = 127.0
+    xi = f32_to_bf16_bits(ints)
+    ci, ai = oracle.quantize_block(xi)
+    assert np.array_equal(ci.astype(np.float32), ints) and np.array_equal(oracle.dequantize_block(ci, ai), xi)
+    # zero block
+    cz, az = oracle.quantize_block(np.zeros((4, 8), dtype=np.uint16))
+    assert not cz.any() and not az.any() and not oracle.dequantize_block(cz, az).any()
