@@ -394,6 +394,61 @@ class CpuSample:
         return flops
 
 
+def int8_cache(pipe, max_over_ranks, bf16_attention_ms, reps=3):
+    """The retained cache stored as int8 codes with per-(block, channel) absmax:
+    quantising compaction of all layers, then per layer dequantisation into a
+    one-layer bf16 buffer followed by that layer's pruned attention."""
+    import torch
+    vark, w = pipe.vark, pipe.w
+    L, B, H, D, S, T = w.layers, w.batch, w.heads, w.head_dim, pipe.S, pipe.T
+    base = pipe.base_host.numpy()
+    total = int(base[-1])
+    dev = pipe.dev
+    kq = torch.empty(max(total, 16), dtype=torch.int8, device=dev)
+    vq = torch.empty_like(kq)
+    ka = torch.empty((L, B, H, S, D), dtype=torch.float32, device=dev)
+    va = torch.empty_like(ka)
+    max_rows = max(int(base[l + 1] - base[l]) // D for l in range(L))
+    kcl = torch.empty(max(max_rows * D, 16), dtype=torch.bfloat16, device=dev)
+    vcl = torch.empty_like(kcl)
+    st = torch.cuda.current_stream()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+
+    def one():
+        ev[0].record(st)
+        vark.vark_quantize_kv_int8(pipe.k, pipe.v, B * H * T * D, L, B, H, pipe.sides, D, pipe.keep, pipe.head_off,
+                                   pipe.seg_off, pipe.layer_base, kq, vq, ka, va)
+        ev[1].record(st)
+        for l in range(L):
+            rows = int(base[l + 1] - base[l]) // D
+            b0 = int(base[l])
+            vark.vark_dequantize_layer_int8(kq[b0:], vq[b0:], ka[l], va[l], rows, B, H, pipe.sides, D,
+                                            pipe.head_off[l], pipe.seg_off[l], kcl, vcl)
+            vark.vark_pruned_attention(pipe.q[l], kcl if rows else None, vcl if rows else None, rows, pipe.k[l],
+                                       pipe.v[l], pipe.sides, -1, pipe.head_off[l], pipe.seg_off[l],
+                                       pipe.past_len[l], pipe.tau[l], pipe.bias[l], pipe.out[l], pipe.status)
+        ev[2].record(st)
+
+    one()
+    torch.cuda.synchronize()
+    tq = ta = 0.0
+    for _ in range(reps):
+        one()
+        torch.cuda.synchronize()
+        tq += ev[0].elapsed_time(ev[1]) / 1e3
+        ta += ev[1].elapsed_time(ev[2]) / 1e3
+    assert int(pipe.status.item()) == 0
+    tq, ta = max_over_ranks(tq / reps), max_over_ranks(ta / reps)
+    bf16_bytes = 2 * 2 * total
+    int8_bytes = 2 * total + 2 * 4 * ka.numel()
+    moved = 2 * total * 2 + 2 * total + 2 * total     # absmax pass reads K,V; code pass reads K,V and writes codes
+    return {"cache_bytes_bf16": bf16_bytes, "cache_bytes_int8": int8_bytes,
+            "cache_ratio": int8_bytes / bf16_bytes, "quantize_ms": tq * 1e3,
+            "quantize_gbs": moved / tq / 1e9,
+            "dequant_plus_attention_ms": ta * 1e3,
+            "bf16_cache_attention_ms": bf16_attention_ms}
+
+
 def ranking_stability(pipe):
     """S-CAS of every layer from two disjoint halves of the calibration seeds,
     compared by vark_rank_stability (Spearman over candidate pairs, Jaccard of
@@ -646,6 +701,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--gen-passes", type=int, default=2)
     ap.add_argument("--stability", type=int, default=1)
+    ap.add_argument("--quant", type=int, default=1)
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -784,6 +840,9 @@ def main():
     # ------------------------------------------------ ranking stability (two disjoint seed halves)
     stab = ranking_stability(pipe) if args.stability else None
 
+    # ------------------------------------------------ int8 retained cache
+    quant = int8_cache(pipe, max_over_ranks, ph["attn"] * 1e3 / K) if args.quant else None
+
     # ------------------------------------------------ generation order (scale by scale)
     gen = None
     if args.gen_passes > 0:
@@ -819,6 +878,7 @@ def main():
                                     "S-CAS, schedule, offsets, compaction, pruned attention of all layers"},
             "pruned_attention_tflops": pruned_tflops, "query_tokens_per_s": qtok_s, "compaction_gbs": comp_gbs,
             "roofline": roof, "kernels": kernels, "generation_order": gen, "ranking_stability": stab,
+            "int8_cache": quant,
             "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches,
             "clocks": clk, "peaks": peaks,
