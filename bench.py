@@ -394,7 +394,7 @@ class CpuSample:
         return flops
 
 
-def int8_cache(pipe, max_over_ranks, bf16_attention_ms, reps=3):
+def int8_cache(pipe, max_over_ranks, bf16_attention_ms, hbm_gbs, reps=3):
     """The retained cache stored as int8 codes with per-(block, channel) absmax:
     quantising compaction of all layers, then per layer dequantisation into a
     one-layer bf16 buffer followed by that layer's pruned attention."""
@@ -428,23 +428,35 @@ def int8_cache(pipe, max_over_ranks, bf16_attention_ms, reps=3):
                                        pipe.v[l], pipe.sides, -1, pipe.head_off[l], pipe.seg_off[l],
                                        pipe.past_len[l], pipe.tau[l], pipe.bias[l], pipe.out[l], pipe.status)
         ev[2].record(st)
+        for l in range(L):     # the dequantisations alone
+            rows = int(base[l + 1] - base[l]) // D
+            b0 = int(base[l])
+            vark.vark_dequantize_layer_int8(kq[b0:], vq[b0:], ka[l], va[l], rows, B, H, pipe.sides, D,
+                                            pipe.head_off[l], pipe.seg_off[l], kcl, vcl)
+        ev[3].record(st)
 
     one()
     torch.cuda.synchronize()
-    tq = ta = 0.0
+    tq = ta = td = 0.0
     for _ in range(reps):
         one()
         torch.cuda.synchronize()
         tq += ev[0].elapsed_time(ev[1]) / 1e3
         ta += ev[1].elapsed_time(ev[2]) / 1e3
+        td += ev[2].elapsed_time(ev[3]) / 1e3
     assert int(pipe.status.item()) == 0
-    tq, ta = max_over_ranks(tq / reps), max_over_ranks(ta / reps)
+    tq, ta, td = max_over_ranks(tq / reps), max_over_ranks(ta / reps), max_over_ranks(td / reps)
     bf16_bytes = 2 * 2 * total
-    int8_bytes = 2 * total + 2 * 4 * ka.numel()
-    moved = 2 * total * 2 + 2 * total + 2 * total     # absmax pass reads K,V; code pass reads K,V and writes codes
+    absmax_bytes = 2 * 4 * ka.numel()
+    int8_bytes = 2 * total + absmax_bytes
+    # algorithmic bytes: quantise = kept bf16 K,V read once + codes and absmax tables written;
+    # dequantise = codes and absmax read + bf16 K,V written
+    q_bytes = bf16_bytes + int8_bytes
     return {"cache_bytes_bf16": bf16_bytes, "cache_bytes_int8": int8_bytes,
             "cache_ratio": int8_bytes / bf16_bytes, "quantize_ms": tq * 1e3,
-            "quantize_gbs": moved / tq / 1e9,
+            "quantize_gbs": q_bytes / tq / 1e9, "quantize_frac_of_hbm": q_bytes / tq / 1e9 / hbm_gbs,
+            "dequantize_ms": td * 1e3, "dequantize_gbs": q_bytes / td / 1e9,
+            "dequantize_frac_of_hbm": q_bytes / td / 1e9 / hbm_gbs,
             "dequant_plus_attention_ms": ta * 1e3,
             "bf16_cache_attention_ms": bf16_attention_ms}
 
@@ -472,6 +484,110 @@ def ranking_stability(pipe):
     sp, jc = vark.vark_rank_stability(sa, sb, pipe.sides, w.budget_bp, w.n_sinks)
     return {"seeds": f"{half} vs {w.n_seeds - half} (disjoint)", "spearman": sp, "drop_jaccard": jc,
             "budget_bp": w.budget_bp, "seconds": time.perf_counter() - t0}
+
+
+def other_configs(rank, device, max_over_ranks, peaks, reps=3):
+    """The two other 1024^2 workloads, timed per kernel with CUDA events
+    (outside the benchmark step):
+    - large_8l: 8 layers x 32 heads, batch 4, 4% budget, 8 calibration seeds:
+      calibration attention, compaction and pruned attention of all layers;
+    - final_scale: the 64x64 scale's 4,096 queries against the 10,521-token
+      cache, budgets {100, 20, 10, 4}% x batch {1, 4, 16, 32}, seed-random
+      retained sets per head; L2 flushed before every timed launch (the
+      small-batch inputs fit in L2)."""
+    import torch
+    import kv_cache_compression_cas_b200 as vark
+    res = {}
+    st = torch.cuda.current_stream()
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+
+    # ---- large_8l
+    w = synth.WORKLOADS["large_8l"]
+    pipe = Pipeline(w, rank, device)
+    ph = {"calib": 0.0, "comp": 0.0, "attn": 0.0}
+    keys = ("t0", "calib", "sched", "offs", "comp", "attn")
+    ev = dict(zip(keys, evs))
+    pipe.step()
+    torch.cuda.synchronize()
+    for _ in range(reps):
+        pipe.step(ev)
+        torch.cuda.synchronize()
+        ph["calib"] += ev["t0"].elapsed_time(ev["calib"]) / 1e3
+        ph["comp"] += ev["offs"].elapsed_time(ev["comp"]) / 1e3
+        ph["attn"] += ev["comp"].elapsed_time(ev["attn"]) / 1e3
+    assert int(pipe.status.item()) == 0
+    for k_ in ph:
+        ph[k_] = max_over_ranks(ph[k_] / reps)
+    keep = pipe.last_keep
+    base = pipe.base_host.numpy()
+    comp_bytes = 2 * 2 * 2 * int(base[-1])
+    pf = pruned_flops(keep, w.sides, w.batch, w.head_dim)
+    res["large_8l"] = {
+        "workload": "8 layers x 32 heads, head_dim 128, 1024^2 scales, batch 4, budget 4%, 8 calibration seeds",
+        "calibration_tflops": pipe.calib_flops / ph["calib"] / 1e12,
+        "calibration_frac_of_bf16_peak": pipe.calib_flops / ph["calib"] / 1e12 / peaks["bf16_tflops_sustained"],
+        "compaction_gbs": comp_bytes / ph["comp"] / 1e9,
+        "compaction_frac_of_hbm": comp_bytes / ph["comp"] / 1e9 / peaks["hbm_gbs"],
+        "pruned_attention_tflops": pf / ph["attn"] / 1e12,
+        "pruned_frac_of_bf16_peak": pf / ph["attn"] / 1e12 / peaks["bf16_tflops_sustained"],
+        "query_tokens_per_s": w.layers * w.batch * pipe.T / ph["attn"],
+        "ms": {k_: v_ * 1e3 for k_, v_ in ph.items()}}
+    del pipe
+    torch.cuda.empty_cache()
+
+    # ---- final_scale sweep
+    w = synth.WORKLOADS["final_scale"]
+    sides, H, D, kq = w.sides, w.heads, w.head_dim, w.query_scale
+    S, T = len(sides), synth.n_tokens(sides)
+    n = [x * x for x in sides]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    tau = torch.from_numpy(synth.gen_tau(w.base_seed, H)).to(device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    rows = []
+    for B in w.extra["batches"]:
+        seed = synth.derive_key(w.base_seed, 0xF5, B, rank)
+        q = randn_bf16((B, H, n[kq], D), seed + 1, device)
+        kd = randn_bf16((B, H, T, D), seed + 2, device)
+        vd = randn_bf16((B, H, T, D), seed + 3, device)
+        out = torch.empty_like(q)
+        for budget in w.extra["budgets_bp"]:
+            keep = synth.random_keep(synth.derive_key(w.base_seed, budget), H, sides, budget, w.n_sinks, kq)
+            keep_d = torch.from_numpy(keep).to(device)
+            ho = torch.empty((1, H), dtype=torch.int32, device=device)
+            so = torch.empty((1, H, S), dtype=torch.int32, device=device)
+            pl = torch.empty((1, H, S), dtype=torch.int32, device=device)
+            lb = torch.empty(2, dtype=torch.int64, device=device)
+            vark.vark_build_offsets(keep_d, sides, B, D, ho, so, pl, lb)
+            total = int(lb[-1].item())
+            kc = torch.empty(max(total, 16), dtype=torch.bfloat16, device=device)
+            vc = torch.empty_like(kc)
+            vark.vark_compact_kv(kd[None], vd[None], B * H * T * D, 1, B, H, sides, D, keep_d, ho, so, lb, kc, vc)
+
+            def launch():
+                vark.vark_pruned_attention(q, kc if total else None, vc if total else None, total // D, kd, vd,
+                                           sides, kq, ho[0], so[0], pl[0], tau, None, out, status)
+            launch()
+            t = 0.0
+            for _ in range(reps):
+                flush.fill_(1)
+                evs[0].record(st)
+                launch()
+                evs[1].record(st)
+                torch.cuda.synchronize()
+                t += evs[0].elapsed_time(evs[1]) / 1e3
+            t = max_over_ranks(t / reps)
+            assert int(status.item()) == 0
+            past = (keep[0, :, :kq].astype(np.float64) * np.array(n[:kq], dtype=np.float64)).sum(axis=1)
+            fl = float((4.0 * B * n[kq] * (past + n[kq]) * D).sum())
+            rows.append({"budget_bp": budget, "batch": B, "tflops": fl / t / 1e12,
+                         "frac_of_bf16_peak": fl / t / 1e12 / peaks["bf16_tflops"],
+                         "query_tokens_per_s": B * n[kq] / t, "ms": t * 1e3})
+        del q, kd, vd, out
+    res["final_scale"] = {"workload": "query scale 12 (4,096 rows) vs the 10,521-token cache, 16 heads, head_dim 128; "
+                                      "fraction against the burst bf16 peak (single launches)", "points": rows}
+    del flush
+    torch.cuda.empty_cache()
+    return res
 
 
 def generation_order(pipe, passes, max_over_ranks, sum_over_ranks):
@@ -644,7 +760,8 @@ def profile_case(case: str, reps: int):
     few GB at most): 'calib' = calibration attention, 4 seeds x 16 heads at
     1024^2; 'pruned' = pruned attention of one layer of the 32-layer
     workload (batch 8, 10% budget schedule); 'compact' = compaction of 4
-    layers of that workload."""
+    layers of that workload; 'quant' = int8 quantising compaction of those 4
+    layers, then the dequantisation of each."""
     import torch
     import kv_cache_compression_cas_b200 as vark
     dev = torch.device("cuda", 0)
@@ -677,6 +794,20 @@ def profile_case(case: str, reps: int):
         reps_c = reps if case == "compact" else 1
         for _ in range(reps_c):
             vark.vark_compact_kv(k, v, B * H * T * D, L, B, H, sides, D, keep_d, ho, so, lb, kc, vc)
+        if case == "quant":
+            kq = torch.empty(max(total, 16), dtype=torch.int8, device=dev)
+            vq = torch.empty_like(kq)
+            ka = torch.empty((L, B, H, S, D), dtype=torch.float32, device=dev)
+            va = torch.empty_like(ka)
+            for _ in range(reps):
+                vark.vark_quantize_kv_int8(k, v, B * H * T * D, L, B, H, sides, D, keep_d, ho, so, lb, kq, vq, ka,
+                                           va)
+            base = lb.cpu().numpy()
+            for _ in range(reps):
+                for l in range(L):
+                    rows = int(base[l + 1] - base[l]) // D
+                    vark.vark_dequantize_layer_int8(kq[int(base[l]):], vq[int(base[l]):], ka[l], va[l], rows, B, H,
+                                                    sides, D, ho[l], so[l], kc, vc)
         if case == "pruned":
             q = randn_bf16((B, H, T, D), 30, dev)
             out = torch.empty_like(q)
@@ -691,7 +822,7 @@ def profile_case(case: str, reps: int):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--profile-case", choices=["calib", "pruned", "compact"], default=None)
+    ap.add_argument("--profile-case", choices=["calib", "pruned", "compact", "quant"], default=None)
     ap.add_argument("--profile-reps", type=int, default=3)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=5)
@@ -702,6 +833,7 @@ def main():
     ap.add_argument("--gen-passes", type=int, default=2)
     ap.add_argument("--stability", type=int, default=1)
     ap.add_argument("--quant", type=int, default=1)
+    ap.add_argument("--other-configs", type=int, default=1)
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -841,7 +973,7 @@ def main():
     stab = ranking_stability(pipe) if args.stability else None
 
     # ------------------------------------------------ int8 retained cache
-    quant = int8_cache(pipe, max_over_ranks, ph["attn"] * 1e3 / K) if args.quant else None
+    quant = int8_cache(pipe, max_over_ranks, ph["attn"] * 1e3 / K, peaks["hbm_gbs"]) if args.quant else None
 
     # ------------------------------------------------ generation order (scale by scale)
     gen = None
@@ -849,6 +981,13 @@ def main():
         del pipe.cq, pipe.ck, pipe.cv
         torch.cuda.empty_cache()
         gen = generation_order(pipe, args.gen_passes, max_over_ranks, sum_over_ranks)
+
+    # ------------------------------------------------ the other 1024^2 workloads (per-kernel figures)
+    others = None
+    if args.other_configs:
+        del pipe
+        torch.cuda.empty_cache()
+        others = other_configs(rank, dev, max_over_ranks, peaks)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -878,7 +1017,7 @@ def main():
                                     "S-CAS, schedule, offsets, compaction, pruned attention of all layers"},
             "pruned_attention_tflops": pruned_tflops, "query_tokens_per_s": qtok_s, "compaction_gbs": comp_gbs,
             "roofline": roof, "kernels": kernels, "generation_order": gen, "ranking_stability": stab,
-            "int8_cache": quant,
+            "int8_cache": quant, "other_configs": others,
             "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches,
             "clocks": clk, "peaks": peaks,

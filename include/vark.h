@@ -342,9 +342,14 @@ int vark_recompact_kv(const uint16_t* kc_old, const uint16_t* vc_old, const int3
 /*
  * vark_quantize_kv_int8 -- device.  Compaction with quantisation: like
  * vark_compact_kv, but writes int8 codes to kq / vq (layer_base[L] bytes each)
- * and the per-(block, channel) absmax to k_absmax / v_absmax.  Reads each kept
- * block twice (absmax pass, code pass).
- * Errors: VARK_E_ARG, VARK_E_SHAPE (D % 8 != 0, D > 512), VARK_E_ALIGN, VARK_E_CUDA.
+ * and the per-(block, channel) absmax to k_absmax / v_absmax.  Each kept block
+ * is read from HBM once (blocks of more than 256 rows are split over the CTAs
+ * of a thread-block cluster, which exchange their partial maxima); the code
+ * pass re-reads the rows from L2.  k, v, kq, vq, k_absmax, v_absmax 16-byte
+ * aligned; layer_stride a multiple of 8.  Non-finite inputs: a NaN in a block
+ * makes that channel's absmax NaN (magnitude bits compare above infinity).
+ * Errors: VARK_E_ARG, VARK_E_SHAPE (D % 8 != 0, D > 512, H > 2048), VARK_E_ALIGN,
+ * VARK_E_CUDA.
  */
 int vark_quantize_kv_int8(const uint16_t* k, const uint16_t* v, int64_t layer_stride,
                           int L, int B, int H, int S, int D, const int32_t* sides,
@@ -360,7 +365,9 @@ int vark_quantize_kv_int8(const uint16_t* k, const uint16_t* v, int64_t layer_st
  *   k_absmax, v_absmax  dev fp32 [B][H][S][D], the layer's absmax tables.
  *   head_off, seg_off   dev int32 [H], [H][S]: the layer's offset tables.
  *   kc, vc        dev bf16 [kc_rows][D] out.
- * Errors: VARK_E_ARG, VARK_E_SHAPE, VARK_E_ALIGN, VARK_E_CUDA.
+ * kq, vq 8-byte aligned; the absmax tables, kc and vc 16-byte aligned.
+ * Errors: VARK_E_ARG, VARK_E_SHAPE (D % 8 != 0, D > 512, H > 4096, kc_rows not a
+ * multiple of B), VARK_E_ALIGN, VARK_E_CUDA.
  */
 int vark_dequantize_layer_int8(const int8_t* kq, const int8_t* vq, const float* k_absmax, const float* v_absmax,
                                int64_t kc_rows, int B, int H, int S, int D, const int32_t* sides,

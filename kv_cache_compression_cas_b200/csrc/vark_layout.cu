@@ -5,8 +5,9 @@
 // scales are generated; the Abstract: allocation is head-specific.
 //
 // Compaction is a pure HBM stream (every retained byte read once and written
-// once, dropped bytes never touched).  Work unit = (layer, head, kept chunk of
-// <= kChunkRows rows of one scale, batch); one persistent grid walks the units.
+// once, dropped bytes never touched).  Work unit = (layer, batch, head, kept
+// chunk of <= kChunkRows rows of one scale), walked in that (memory) order by
+// one persistent grid.
 // Each CTA first builds, in shared memory, the prefix of kept chunks over
 // (layer, head) for its layer group, so a unit is found by one binary search
 // and a walk over at most S scales.  Copies are 16-byte vectors, coalesced,
@@ -85,7 +86,7 @@ struct CompactParams {
   const int64_t* src_layer_base;
 };
 
-__global__ void __launch_bounds__(kCompactThreads) compact_kernel(
+__global__ void __launch_bounds__(kCompactThreads, 4) compact_kernel(
     const uint4* __restrict__ k, const uint4* __restrict__ v, CompactParams p, const uint8_t* __restrict__ keep,
     const int32_t* __restrict__ head_off, const int32_t* __restrict__ seg_off, const int64_t* __restrict__ layer_base,
     uint4* __restrict__ kc, uint4* __restrict__ vc) {
@@ -149,10 +150,21 @@ __global__ void __launch_bounds__(kCompactThreads) compact_kernel(
   const int vec_per_row = p.D / 8;  // 16-byte vectors per row
 
   for (int64_t g = blockIdx.x; g < units; g += gridDim.x) {
-    const int b = int(g % p.B);
-    const int32_t c = int32_t(g / p.B);
-    // (layer, head) with chunk_prefix[i] <= c < chunk_prefix[i+1]
-    int lo = 0, hi = nlh;
+    // Units in memory order (layer, batch, head, kept chunk): the CTAs in flight
+    // read and write neighbouring addresses.  Layer: the last li with
+    // B * chunk_prefix[li * H] <= g (empty layers are skipped by taking the last).
+    int la = 0, lz = p.nl;
+    while (lz - la > 1) {
+      const int mid = (la + lz) >> 1;
+      if (int64_t(chunk_prefix[mid * H]) * p.B <= g) la = mid; else lz = mid;
+    }
+    const int32_t c0 = chunk_prefix[la * H];
+    const int32_t C = chunk_prefix[(la + 1) * H] - c0;
+    const int64_t r = g - int64_t(c0) * p.B;
+    const int b = int(r / C);
+    const int32_t c = c0 + int32_t(r % C);
+    // (layer, head) with chunk_prefix[i] <= c < chunk_prefix[i+1], inside layer la
+    int lo = la * H, hi = (la + 1) * H;
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
       if (chunk_prefix[mid] <= c) lo = mid; else hi = mid;
@@ -325,56 +337,50 @@ extern "C" int vark_recompact_kv(const uint16_t* kc_old, const uint16_t* vc_old,
                        static_cast<cudaStream_t>(stream));
 }
 
+
 // ---------------------------------------------------------------- int8 quantised retained cache
 // [VAR-Q] summary page: groups indexed by (block, channel), block boundaries
 // given by the generation loop, composable with eviction.  Here a block is one
 // retained scale of one (layer, batch, head); every channel d of it has one
 // absmax a; codes are rint(x / (a / 127)) clamped to [-127, 127] (IEEE fp32
 // division, round half to even); x' = code * (a / 127).
+//
+// Quantisation reads every kept byte from HBM once.  A unit is one block of
+// one tensor (K or V).  A block of at most kSmallRows rows (256 KB at D = 128)
+// belongs to one CTA:
+// a strided pass takes the channel maxima, a second pass over the same rows
+// (still in L2) writes the codes.  A larger block is split over the
+// kQuantCluster CTAs of a thread-block cluster: each CTA reduces its slice,
+// the CTAs exchange partial maxima through distributed shared memory, then
+// each writes the codes of its slice.  Channel maxima are taken on the bf16
+// magnitude bits (non-negative bf16 values order like their bit patterns), two
+// channels per 32-bit word.  Every absmax entry is written exactly once.
 
 namespace vark {
 
-constexpr int kQuantThreads = 256;
+constexpr int kQuantThreads = 128;
+constexpr int kQuantCluster = 8;
+constexpr int kQuantGroupLH = 2048;  // (layer, head) pairs per launch group
+constexpr int kSmallRows = 1024;
+constexpr int kQuantMaxD = 512;
 
 struct QuantParams {
-  CompactParams c;          // layout and unit walk (dense source)
-  int mode;                 // 0: absmax pass, 1: quantise pass
-  int64_t scale_stride_l;   // B*H*S*D
+  ScaleTable sc;
+  uint32_t big_mask;        // scales with n_s > kSmallRows
+  int l0, nl;               // layer group [l0, l0 + nl)
+  int L, B, H, D;
+  int64_t layer_stride;     // elements between source layers
 };
 
-// One unit = (layer, head, kept chunk, batch) as in compact_kernel.  Every
-// thread owns one channel-pair column of the chunk (D/2 columns) and strides
-// over its rows.
-__global__ void __launch_bounds__(kQuantThreads) quant_kernel(
-    const uint16_t* __restrict__ k, const uint16_t* __restrict__ v, QuantParams q, const uint8_t* __restrict__ keep,
-    const int32_t* __restrict__ head_off, const int32_t* __restrict__ seg_off, const int64_t* __restrict__ layer_base,
-    int8_t* __restrict__ kq, int8_t* __restrict__ vq, float* __restrict__ ka, float* __restrict__ va) {
-  const CompactParams& p = q.c;
-  __shared__ int32_t chunk_prefix[kMaxGroupLH + 1];
-  __shared__ uint32_t keep_mask[kMaxGroupLH];
-  __shared__ int32_t warp_tot[kQuantThreads / 32];
-  const int S = p.sc.S;
-  const int H = p.H;
-  const int nlh = p.nl * H;
-  const int lh0 = p.l0 * H;
-  for (int i = threadIdx.x; i < nlh; i += kQuantThreads) {
-    const uint8_t* kp = keep + int64_t(lh0 + i) * S;
-    uint32_t m = 0;
-    int32_t c = 0;
-    for (int s = 0; s < S; ++s)
-      if (kp[s] && p.chunks[s] > 0) {
-        m |= 1u << s;
-        c += p.chunks[s];
-      }
-    keep_mask[i] = m;
-    chunk_prefix[i] = c;
-  }
-  __syncthreads();
-  constexpr int kPer = (kMaxGroupLH + kQuantThreads - 1) / kQuantThreads;
+// Exclusive scan of a[0, n) in shared memory by the whole block (kThreads
+// threads, each owning a contiguous segment); a[n] receives the total.
+template <int kThreads, int kMaxN>
+__device__ __forceinline__ void block_exclusive_scan(int32_t* a, int n, int32_t* warp_tot) {
+  constexpr int kPer = (kMaxN + kThreads - 1) / kThreads;
   const int seg0 = threadIdx.x * kPer;
   int32_t my_total = 0;
   for (int u = 0; u < kPer; ++u)
-    if (seg0 + u < nlh) my_total += chunk_prefix[seg0 + u];
+    if (seg0 + u < n) my_total += a[seg0 + u];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int32_t incl = my_total;
 #pragma unroll
@@ -386,140 +392,373 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(
   __syncthreads();
   int32_t warp_base = 0, grand = 0;
 #pragma unroll
-  for (int w = 0; w < kQuantThreads / 32; ++w) {
+  for (int w = 0; w < kThreads / 32; ++w) {
     if (w < warp) warp_base += warp_tot[w];
     grand += warp_tot[w];
   }
   int32_t run = warp_base + incl - my_total;
   for (int u = 0; u < kPer; ++u)
-    if (seg0 + u < nlh) {
-      const int32_t c = chunk_prefix[seg0 + u];
-      chunk_prefix[seg0 + u] = run;
+    if (seg0 + u < n) {
+      const int32_t c = a[seg0 + u];
+      a[seg0 + u] = run;
       run += c;
     }
-  if (threadIdx.x == 0) chunk_prefix[nlh] = grand;
+  if (threadIdx.x == 0) a[n] = grand;
   __syncthreads();
+}
 
-  const int64_t units = int64_t(grand) * p.B;
-  const int cols = p.D / 2;                          // channel pairs
-  const int col = threadIdx.x % cols;
-  const int rstep = kQuantThreads / cols;
-  const int rofs = threadIdx.x / cols;
-  for (int64_t g = blockIdx.x; g < units; g += gridDim.x) {
-    const int b = int(g % p.B);
-    const int32_t c = int32_t(g / p.B);
-    int lo = 0, hi = nlh;
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (chunk_prefix[mid] <= c) lo = mid; else hi = mid;
+struct QBlock {
+  int l, h, s, b, t;        // t: 0 = K, 1 = V
+};
+
+// Unit g of one size class: blocks of the class are numbered in memory order
+// (layer, batch, head, kept scale), K and V of a block adjacent.
+__device__ __forceinline__ QBlock decode_block(int64_t g, const int32_t* prefix, const uint32_t* masks,
+                                               uint32_t cls, const QuantParams& p) {
+  const int H = p.H;
+  const int64_t two_b = 2 * int64_t(p.B);
+  int la = 0, lz = p.nl;                      // last layer whose first unit is <= g
+  while (lz - la > 1) {
+    const int mid = (la + lz) >> 1;
+    if (int64_t(prefix[mid * H]) * two_b <= g) la = mid; else lz = mid;
+  }
+  const int32_t c0 = prefix[la * H];
+  const int64_t C2 = 2 * int64_t(prefix[(la + 1) * H] - c0);   // units per batch entry of the layer
+  const int64_t r = g - int64_t(c0) * two_b;
+  const int32_t rem = int32_t(r % C2);
+  const int32_t c = c0 + (rem >> 1);
+  int lo = la * H, hi = (la + 1) * H;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (prefix[mid] <= c) lo = mid; else hi = mid;
+  }
+  uint32_t m = masks[lo] & cls;
+  for (int32_t j = c - prefix[lo]; j > 0; --j) m &= m - 1;   // drop the j lowest kept scales
+  QBlock q;
+  q.s = __ffs(m) - 1;
+  q.l = p.l0 + la;
+  q.h = lo - la * H;
+  q.b = int(r / C2);
+  q.t = rem & 1;
+  return q;
+}
+
+// Per-channel maximum of |x| over 8 bf16 channels, as magnitude bits.
+__device__ __forceinline__ void absmax8(uint32_t (&acc)[4], const uint4& x) {
+  acc[0] = __vmaxu2(acc[0], x.x & 0x7FFF7FFFu);
+  acc[1] = __vmaxu2(acc[1], x.y & 0x7FFF7FFFu);
+  acc[2] = __vmaxu2(acc[2], x.z & 0x7FFF7FFFu);
+  acc[3] = __vmaxu2(acc[3], x.w & 0x7FFF7FFFu);
+}
+
+// Channel scale: sc = a / 127 (IEEE), and rc = RN(1 / sc) when the product
+// path is usable (sc normal and not tiny), else 0 (always divide).
+struct QScale {
+  float sc, rc;
+};
+
+__device__ __forceinline__ QScale make_qscale(float a) {
+  QScale q;
+  q.sc = a / 127.f;
+  q.rc = (q.sc >= 0x1p-100f && q.sc <= 0x1p100f) ? __frcp_rn(q.sc) : 0.f;
+  return q;
+}
+
+// Codes of 8 channels: rint(x / sc) with x / sc the IEEE quotient, clamped to
+// [-127, 127].  |x| <= a and sc = RN(a / 127) give |x / sc| <= 127 (1 + 2^-24),
+// so the clamp never binds for finite inputs and is left out.  The product
+// t = x * rc (rc = RN(1 / sc)) differs from the quotient by at most
+// |t| * 1.5 * 2^-23 (two roundings of relative 2^-24, plus the quotient's own
+// half ulp), so rint(t) = rint(quotient) unless t lies within that distance of
+// a half-integer.  Elements within |t| * 2^-20 of one (ties x = a / 2 are
+// common in bf16 data) take the exact division instead.
+__device__ __forceinline__ float lo_bf16(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float hi_bf16(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint32_t pack4_s8(float r0, float r1, float r2, float r3) {
+  const uint32_t c0 = uint32_t(__float2int_rn(r0)), c1 = uint32_t(__float2int_rn(r1));
+  const uint32_t c2 = uint32_t(__float2int_rn(r2)), c3 = uint32_t(__float2int_rn(r3));
+  return __byte_perm(__byte_perm(c0, c1, 0x0040), __byte_perm(c2, c3, 0x0040), 0x5410);
+}
+
+__device__ __forceinline__ uint2 codes8(const uint4& x, const float (&sc)[8], const float (&rc)[8], bool force) {
+  const float v[8] = {lo_bf16(x.x), hi_bf16(x.x), lo_bf16(x.y), hi_bf16(x.y),
+                      lo_bf16(x.z), hi_bf16(x.z), lo_bf16(x.w), hi_bf16(x.w)};
+  float r[8], d[8];   // d > 1/2: the product lies within |t| * 2^-20 of a half-integer
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float t = v[j] * rc[j];
+    r[j] = rintf(t);
+    d[j] = fmaf(fabsf(t), 0x1p-20f, fabsf(t - r[j]));
+  }
+  const float dmax = fmaxf(fmaxf(fmaxf(d[0], d[1]), fmaxf(d[2], d[3])), fmaxf(fmaxf(d[4], d[5]), fmaxf(d[6], d[7])));
+  if (force || dmax > 0.5f) {   // rare: decide the flagged elements by the exact quotient
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (force || d[j] > 0.5f) r[j] = sc[j] == 0.f ? 0.f : rintf(__fdiv_rn(v[j], sc[j]));
+  }
+  uint2 o;
+  o.x = pack4_s8(r[0], r[1], r[2], r[3]);
+  o.y = pack4_s8(r[4], r[5], r[6], r[7]);
+  return o;
+}
+
+__global__ void __cluster_dims__(kQuantCluster, 1, 1) __launch_bounds__(kQuantThreads, 6) quant_kernel(
+    const uint4* __restrict__ k, const uint4* __restrict__ v, QuantParams p, const uint8_t* __restrict__ keep,
+    const int32_t* __restrict__ head_off, const int32_t* __restrict__ seg_off, const int64_t* __restrict__ layer_base,
+    int8_t* __restrict__ kq, int8_t* __restrict__ vq, float* __restrict__ ka, float* __restrict__ va) {
+  __shared__ int32_t big_prefix[kQuantGroupLH + 1];
+  __shared__ int32_t small_prefix[kQuantGroupLH + 1];
+  __shared__ uint32_t keep_mask[kQuantGroupLH];
+  __shared__ int32_t warp_tot[kQuantThreads / 32];
+  __shared__ __align__(16) uint32_t red[kQuantThreads * 4];
+  __shared__ uint32_t part[2][kQuantMaxD / 2];   // read by the other CTAs of the cluster
+  __shared__ uint32_t fin[kQuantMaxD / 2];
+  __shared__ __align__(16) float fin_sc[kQuantMaxD];   // a / 127 per channel
+  __shared__ __align__(16) float fin_rc[kQuantMaxD];   // RN(1 / (a / 127)), or 0: divide
+
+  const int S = p.sc.S, H = p.H, D = p.D, B = p.B;
+  const int nlh = p.nl * H;
+  const int lh0 = p.l0 * H;
+  for (int i = threadIdx.x; i < nlh; i += kQuantThreads) {
+    const uint8_t* kp = keep + int64_t(lh0 + i) * S;
+    uint32_t m = 0;
+    for (int s = 0; s < S; ++s)
+      if (kp[s]) m |= 1u << s;
+    keep_mask[i] = m;
+    big_prefix[i] = __popc(m & p.big_mask);
+    small_prefix[i] = __popc(m & ~p.big_mask);
+  }
+  __syncthreads();
+  block_exclusive_scan<kQuantThreads, kQuantGroupLH>(big_prefix, nlh, warp_tot);
+  block_exclusive_scan<kQuantThreads, kQuantGroupLH>(small_prefix, nlh, warp_tot);
+
+  const int64_t n_big = int64_t(big_prefix[nlh]) * 2 * B;
+  const int64_t n_small = int64_t(small_prefix[nlh]) * 2 * B;
+  const int64_t n_units = n_big + (n_small + kQuantCluster - 1) / kQuantCluster;
+  const uint32_t rank = cluster_ctarank();
+  const int cv_n = D / 8;                         // 16-byte vectors per row
+  const int nrg = kQuantThreads / cv_n;           // row groups
+  const bool active = threadIdx.x < nrg * cv_n;
+  const int cv = threadIdx.x % cv_n;
+  const int rg = threadIdx.x / cv_n;
+  const int dw = D / 2;                           // channel-pair words per row
+  int parity = 0;
+
+  // Units are taken cluster-wide: big blocks first, then packs of kQuantCluster
+  // small blocks (one per CTA).  Every CTA of a cluster runs the same
+  // iterations, so the cluster barriers below match up.
+  for (int64_t u = cluster_id_x(); u < n_units; u += cluster_count_x()) {
+    const bool big = u < n_big;
+    const int64_t g = big ? u : (u - n_big) * kQuantCluster + rank;
+    const bool have = big || g < n_small;
+    QBlock q{0, 0, 0, 0, 0};
+    int32_t r_lo = 0, r_hi = 0;
+    if (have) {
+      q = big ? decode_block(g, big_prefix, keep_mask, p.big_mask, p)
+              : decode_block(g, small_prefix, keep_mask, ~p.big_mask, p);
+      const int32_t n = p.sc.n[q.s];
+      if (big) {
+        const int32_t per = (n + kQuantCluster - 1) / kQuantCluster;
+        r_lo = min(n, int32_t(rank) * per);
+        r_hi = min(n, r_lo + per);
+      } else {
+        r_hi = n;
+      }
     }
-    const int i = lo;
-    int32_t j = c - chunk_prefix[i];
-    const uint32_t m = keep_mask[i];
-    int s = 0;
-    for (; s < S; ++s)
-      if (m >> s & 1u) {
-        if (j < p.chunks[s]) break;
-        j -= p.chunks[s];
+    // this CTA's first row of the block; rows below are 32-bit offsets (a block has at most 2^31 / D rows)
+    const uint4* src = (q.t ? v : k) +
+                       (int64_t(q.l) * p.layer_stride + ((int64_t(q.b) * H + q.h) * p.sc.T + p.sc.off[q.s]) * D) / 8 +
+                       int64_t(r_lo) * cv_n + cv;
+    const int32_t nr = r_hi - r_lo;
+    // 1. channel maxima of this CTA's rows (normal caching: pass 2 re-reads them)
+    uint32_t acc[4] = {0u, 0u, 0u, 0u};
+    if (active) {
+      int32_t r = rg;
+      for (; r + 7 * nrg < nr; r += 8 * nrg) {
+        uint4 x[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = __ldg(src + (r + e * nrg) * cv_n);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) absmax8(acc, x[e]);
       }
-    const int l = p.l0 + i / H;
-    const int h = i % H;
-    const int32_t r0 = j * kChunkRows;
-    const int32_t nrows = min(kChunkRows, p.sc.n[s] - r0);
-    const int64_t src_row0 = (int64_t(b) * H + h) * p.src_rows + p.src_off[s] + r0;
-    const uint16_t* ks = k + int64_t(l) * p.layer_stride + src_row0 * p.D + 2 * col;
-    const uint16_t* vs = v + int64_t(l) * p.layer_stride + src_row0 * p.D + 2 * col;
-    float* kav = ka + int64_t(l) * q.scale_stride_l + ((int64_t(b) * H + h) * S + s) * p.D + 2 * col;
-    float* vav = va + int64_t(l) * q.scale_stride_l + ((int64_t(b) * H + h) * S + s) * p.D + 2 * col;
-    if (q.mode == 0) {
-      float mk0 = 0.f, mk1 = 0.f, mv0 = 0.f, mv1 = 0.f;
-      for (int r = rofs; r < nrows; r += rstep) {
-        const uint32_t wk = *reinterpret_cast<const uint32_t*>(ks + int64_t(r) * p.D);
-        const uint32_t wv = *reinterpret_cast<const uint32_t*>(vs + int64_t(r) * p.D);
-        mk0 = fmaxf(mk0, fabsf(__uint_as_float(wk << 16)));
-        mk1 = fmaxf(mk1, fabsf(__uint_as_float(wk & 0xFFFF0000u)));
-        mv0 = fmaxf(mv0, fabsf(__uint_as_float(wv << 16)));
-        mv1 = fmaxf(mv1, fabsf(__uint_as_float(wv & 0xFFFF0000u)));
+      for (; r < nr; r += nrg) absmax8(acc, __ldg(src + r * cv_n));
+      *reinterpret_cast<uint4*>(&red[threadIdx.x * 4]) = make_uint4(acc[0], acc[1], acc[2], acc[3]);
+    }
+    __syncthreads();
+    // channel pairs x = threadIdx.x, threadIdx.x + kQuantThreads, ... (below dw)
+    for (int x = threadIdx.x; x < dw; x += kQuantThreads) {
+      uint32_t w = 0;
+      for (int e = 0; e < nrg; ++e) w = __vmaxu2(w, red[e * dw + x]);
+      if (big) part[parity][x] = w; else fin[x] = w;
+    }
+    if (big) {
+      cluster_sync_all();
+      for (int x = threadIdx.x; x < dw; x += kQuantThreads) {
+        const uint32_t a = smem_u32(&part[parity][x]);
+        uint32_t w = 0;
+        for (uint32_t c = 0; c < kQuantCluster; ++c)
+          w = __vmaxu2(w, __float_as_uint(ld_shared_cluster_f32(map_shared_rank(a, c))));
+        fin[x] = w;
       }
-      // non-negative floats order like their bit patterns
-      atomicMax(reinterpret_cast<unsigned int*>(kav), __float_as_uint(mk0));
-      atomicMax(reinterpret_cast<unsigned int*>(kav + 1), __float_as_uint(mk1));
-      atomicMax(reinterpret_cast<unsigned int*>(vav), __float_as_uint(mv0));
-      atomicMax(reinterpret_cast<unsigned int*>(vav + 1), __float_as_uint(mv1));
-    } else {
-      const float sk0 = kav[0] / 127.f, sk1 = kav[1] / 127.f;
-      const float sv0 = vav[0] / 127.f, sv1 = vav[1] / 127.f;
-      const int64_t R_l = (layer_base[l + 1] - layer_base[l]) / (int64_t(p.B) * p.D);
-      const int64_t dst_row0 = int64_t(b) * R_l + head_off[l * H + h] + seg_off[(l * H + h) * S + s] + r0;
-      int8_t* kd = kq + layer_base[l] + dst_row0 * p.D + 2 * col;
-      int8_t* vd = vq + layer_base[l] + dst_row0 * p.D + 2 * col;
-      auto code = [](float x, float sc) -> int {
-        if (sc == 0.f) return 0;
-        const float t = rintf(__fdiv_rn(x, sc));
-        return int(fminf(fmaxf(t, -127.f), 127.f));
-      };
-      for (int r = rofs; r < nrows; r += rstep) {
-        const uint32_t wk = *reinterpret_cast<const uint32_t*>(ks + int64_t(r) * p.D);
-        const uint32_t wv = *reinterpret_cast<const uint32_t*>(vs + int64_t(r) * p.D);
-        const int k0 = code(__uint_as_float(wk << 16), sk0), k1 = code(__uint_as_float(wk & 0xFFFF0000u), sk1);
-        const int v0 = code(__uint_as_float(wv << 16), sv0), v1 = code(__uint_as_float(wv & 0xFFFF0000u), sv1);
-        *reinterpret_cast<uint16_t*>(kd + int64_t(r) * p.D) = uint16_t((k0 & 0xFF) | ((k1 & 0xFF) << 8));
-        *reinterpret_cast<uint16_t*>(vd + int64_t(r) * p.D) = uint16_t((v0 & 0xFF) | ((v1 & 0xFF) << 8));
+      parity ^= 1;   // the next big unit writes the other buffer while peers may still read this one
+    }
+    for (int x = threadIdx.x; x < dw; x += kQuantThreads) {   // the pair's scales, once per unit
+      const uint32_t w = fin[x];
+      const QScale q0 = make_qscale(lo_bf16(w)), q1 = make_qscale(hi_bf16(w));
+      fin_sc[2 * x] = q0.sc;
+      fin_sc[2 * x + 1] = q1.sc;
+      fin_rc[2 * x] = q0.rc;
+      fin_rc[2 * x + 1] = q1.rc;
+    }
+    __syncthreads();
+    if (!have) continue;
+    // 2. codes of this CTA's rows
+    if (active && nr > 0) {
+      float sc[8], rc[8];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float4 a = *reinterpret_cast<const float4*>(&fin_sc[cv * 8 + 4 * e]);
+        const float4 b = *reinterpret_cast<const float4*>(&fin_rc[cv * 8 + 4 * e]);
+        sc[4 * e] = a.x; sc[4 * e + 1] = a.y; sc[4 * e + 2] = a.z; sc[4 * e + 3] = a.w;
+        rc[4 * e] = b.x; rc[4 * e + 1] = b.y; rc[4 * e + 2] = b.z; rc[4 * e + 3] = b.w;
+      }
+      bool force = false;   // a channel whose scale is non-zero but has no usable reciprocal
+#pragma unroll
+      for (int j = 0; j < 8; ++j) force |= sc[j] != 0.f && rc[j] == 0.f;
+      const int64_t R_l = (layer_base[q.l + 1] - layer_base[q.l]) / (int64_t(B) * D);
+      const int64_t row0 =
+          int64_t(q.b) * R_l + head_off[q.l * H + q.h] + seg_off[(int64_t(q.l) * H + q.h) * S + q.s];
+      uint2* dst = reinterpret_cast<uint2*>((q.t ? vq : kq) + layer_base[q.l] + (row0 + r_lo) * D) + cv;
+      int32_t r = rg;
+      for (; r + 3 * nrg < nr; r += 4 * nrg) {
+        uint4 x[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[e] = __ldcs(src + (r + e * nrg) * cv_n);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dst[(r + e * nrg) * cv_n] = codes8(x[e], sc, rc, force);
+      }
+      for (; r < nr; r += nrg) dst[r * cv_n] = codes8(__ldcs(src + r * cv_n), sc, rc, force);
+    }
+    // the block's absmax entries: once per block
+    if (!big || rank == 0) {
+      float* ab = (q.t ? va : ka) + ((((int64_t(q.l) * B + q.b) * H + q.h) * S) + q.s) * D;
+      for (int c = threadIdx.x; c < D; c += kQuantThreads) {
+        const uint32_t w = fin[c >> 1];
+        ab[c] = (c & 1) ? hi_bf16(w) : lo_bf16(w);
       }
     }
   }
+  cluster_sync_all();   // no CTA leaves while a peer may still read its partial maxima
 }
 
-// Dequantisation of one layer: one warp per row of the layer's compacted
-// block, 4 channels per lane; the row's (b, h, scale) comes from the layer's
-// offset tables, x' = code * (absmax / 127) rounded to bf16.
+// Dequantisation of one layer.  Unit = (batch, head, kept scale, chunk of at
+// most kDeqRows rows), in that (memory) order; each thread keeps the scales of
+// its 8 channels for the unit and streams rows, four at a time: 8-byte code
+// loads, 16-byte bf16 stores (normal caching: the attention that follows reads
+// them).
+constexpr int kDeqRows = 128;
+constexpr int kDeqThreads = 256;
+constexpr int kDeqMaxH = 4096;
+
 struct DequantParams {
   ScaleTable sc;
   int B, H, D;
-  int64_t rows;            // B * R_l
+  int64_t R;               // rows per batch entry of the layer
 };
 
-__global__ void __launch_bounds__(256) dequant_kernel(const int8_t* __restrict__ kq, const int8_t* __restrict__ vq,
-                                                      const float* __restrict__ ka, const float* __restrict__ va,
-                                                      DequantParams p, const int32_t* __restrict__ head_off,
-                                                      const int32_t* __restrict__ seg_off, uint16_t* __restrict__ kc,
-                                                      uint16_t* __restrict__ vc) {
-  const int lane = threadIdx.x & 31;
-  const int64_t warps = int64_t(gridDim.x) * (blockDim.x / 32);
-  const int64_t R = p.rows / p.B;
-  const int S = p.sc.S;
-  for (int64_t row = int64_t(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5); row < p.rows; row += warps) {
-    const int b = int(row / R);
-    const int64_t rr = row - int64_t(b) * R;
-    int lo = 0, hi = p.H;                 // head: last h with head_off[h] <= rr
+__global__ void __launch_bounds__(kDeqThreads, 3) dequant_kernel(const uint2* __restrict__ kq,
+                                                              const uint2* __restrict__ vq,
+                                                              const float* __restrict__ ka,
+                                                              const float* __restrict__ va, DequantParams p,
+                                                              const int32_t* __restrict__ head_off,
+                                                              const int32_t* __restrict__ seg_off,
+                                                              uint4* __restrict__ kc, uint4* __restrict__ vc) {
+  __shared__ int32_t prefix[kDeqMaxH + 1];
+  __shared__ uint32_t masks[kDeqMaxH];
+  __shared__ int32_t warp_tot[kDeqThreads / 32];
+  const int S = p.sc.S, H = p.H, D = p.D, B = p.B;
+  for (int h = threadIdx.x; h < H; h += kDeqThreads) {
+    uint32_t m = 0;
+    int32_t c = 0;
+    for (int s = 0; s < S; ++s)
+      if (seg_off[h * S + s] >= 0) {
+        m |= 1u << s;
+        c += (p.sc.n[s] + kDeqRows - 1) / kDeqRows;
+      }
+    masks[h] = m;
+    prefix[h] = c;
+  }
+  __syncthreads();
+  block_exclusive_scan<kDeqThreads, kDeqMaxH>(prefix, H, warp_tot);
+  const int32_t C = prefix[H];                 // chunks per batch entry of the layer
+  const int64_t units = int64_t(C) * B;
+  const int cv_n = D / 8;
+  const int nrg = kDeqThreads / cv_n;
+  if (threadIdx.x >= nrg * cv_n) return;   // no block-wide barrier follows
+  const int cv = threadIdx.x % cv_n;
+  const int rg = threadIdx.x / cv_n;
+  auto expand = [](uint2 w, const float (&sc)[8]) {
+    auto x = [](uint32_t u, int i) { return float(int8_t((u >> (8 * i)) & 0xFFu)); };
+    uint4 o;
+    o.x = pack_bf16x2(x(w.x, 0) * sc[0], x(w.x, 1) * sc[1]);
+    o.y = pack_bf16x2(x(w.x, 2) * sc[2], x(w.x, 3) * sc[3]);
+    o.z = pack_bf16x2(x(w.y, 0) * sc[4], x(w.y, 1) * sc[5]);
+    o.w = pack_bf16x2(x(w.y, 2) * sc[6], x(w.y, 3) * sc[7]);
+    return o;
+  };
+  // units in memory order (batch, head, kept chunk)
+  for (int64_t g = blockIdx.x; g < units; g += gridDim.x) {
+    const int b = int(g / C);
+    const int32_t c = int32_t(g % C);
+    int lo = 0, hi = H;
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
-      if (head_off[mid] <= rr) lo = mid; else hi = mid;
+      if (prefix[mid] <= c) lo = mid; else hi = mid;
     }
-    // heads that keep nothing share head_off with the next head: take the last
-    while (lo + 1 < p.H && head_off[lo + 1] <= rr) ++lo;
     const int h = lo;
-    const int64_t within = rr - head_off[h];
-    int sc = -1;
-    for (int s = 0; s < S; ++s) {
-      const int32_t so = seg_off[h * S + s];
-      if (so >= 0 && within >= so && within < so + p.sc.n[s]) sc = s;
+    int32_t j = c - prefix[h];
+    const uint32_t m = masks[h];
+    int s = 0;
+    for (; s < S; ++s)
+      if (m >> s & 1u) {
+        const int32_t ch = (p.sc.n[s] + kDeqRows - 1) / kDeqRows;
+        if (j < ch) break;
+        j -= ch;
+      }
+    const int32_t r0 = j * kDeqRows;
+    const int32_t nrows = min(kDeqRows, p.sc.n[s] - r0);
+    const int64_t row0 = int64_t(b) * p.R + head_off[h] + seg_off[h * S + s] + r0;
+    const int64_t arow = ((int64_t(b) * H + h) * S + s) * D + cv * 8;
+    float sk[8], sv[8];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const float4 a = *reinterpret_cast<const float4*>(ka + arow + 4 * e);
+      const float4 bq = *reinterpret_cast<const float4*>(va + arow + 4 * e);
+      sk[4 * e] = a.x / 127.f; sk[4 * e + 1] = a.y / 127.f; sk[4 * e + 2] = a.z / 127.f; sk[4 * e + 3] = a.w / 127.f;
+      sv[4 * e] = bq.x / 127.f; sv[4 * e + 1] = bq.y / 127.f; sv[4 * e + 2] = bq.z / 127.f; sv[4 * e + 3] = bq.w / 127.f;
     }
-    if (sc < 0) continue;
-    const int64_t arow = ((int64_t(b) * p.H + h) * S + sc) * p.D;
-    for (int d = lane * 4; d < p.D; d += 128) {
-      const uint32_t ck = *reinterpret_cast<const uint32_t*>(kq + row * p.D + d);
-      const uint32_t cv = *reinterpret_cast<const uint32_t*>(vq + row * p.D + d);
-      const float4 ak = *reinterpret_cast<const float4*>(ka + arow + d);
-      const float4 av = *reinterpret_cast<const float4*>(va + arow + d);
-      auto x = [](uint32_t w, int i) { return float(int8_t((w >> (8 * i)) & 0xFF)); };
-      uint2 ok, ov;
-      ok.x = pack_bf16x2(x(ck, 0) * (ak.x / 127.f), x(ck, 1) * (ak.y / 127.f));
-      ok.y = pack_bf16x2(x(ck, 2) * (ak.z / 127.f), x(ck, 3) * (ak.w / 127.f));
-      ov.x = pack_bf16x2(x(cv, 0) * (av.x / 127.f), x(cv, 1) * (av.y / 127.f));
-      ov.y = pack_bf16x2(x(cv, 2) * (av.z / 127.f), x(cv, 3) * (av.w / 127.f));
-      *reinterpret_cast<uint2*>(kc + row * p.D + d) = ok;
-      *reinterpret_cast<uint2*>(vc + row * p.D + d) = ov;
+    const int64_t e0 = row0 * cv_n + cv;
+    int32_t r = rg;
+    for (; r + 3 * nrg < nrows; r += 4 * nrg) {     // 4 rows' loads in flight, then the stores
+      uint2 ck[4], cw[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        ck[u] = __ldcs(kq + e0 + int64_t(r + u * nrg) * cv_n);
+        cw[u] = __ldcs(vq + e0 + int64_t(r + u * nrg) * cv_n);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        kc[e0 + int64_t(r + u * nrg) * cv_n] = expand(ck[u], sk);
+        vc[e0 + int64_t(r + u * nrg) * cv_n] = expand(cw[u], sv);
+      }
+    }
+    for (; r < nrows; r += nrg) {
+      const int64_t e = e0 + int64_t(r) * cv_n;
+      const uint2 ck = __ldcs(kq + e);
+      const uint2 cw = __ldcs(vq + e);
+      kc[e] = expand(ck, sk);
+      vc[e] = expand(cw, sv);
     }
   }
 }
@@ -535,12 +774,14 @@ extern "C" int vark_quantize_kv_int8(const uint16_t* k, const uint16_t* v, int64
   if (!k || !v || !keep || !head_off || !seg_off || !layer_base || !kq || !vq || !k_absmax || !v_absmax)
     return VARK_E_ARG;
   QuantParams q;
-  CompactParams& p = q.c;
-  int rc = make_scale_table(S, sides, &p.sc);
+  int rc = make_scale_table(S, sides, &q.sc);
   if (rc) return rc;
-  if (L < 1 || H < 1 || B < 1 || D < 8 || D % 8 != 0 || D > 512) return VARK_E_SHAPE;
-  if (H > kMaxGroupLH) return VARK_E_SHAPE;
-  if (layer_stride < int64_t(B) * H * p.sc.T * D) return VARK_E_ARG;
+  if (L < 1 || H < 1 || B < 1 || D < 8 || D % 8 != 0 || D > kQuantMaxD) return VARK_E_SHAPE;
+  if (H > kQuantGroupLH) return VARK_E_SHAPE;
+  for (int s = 0; s < S; ++s)   // rows of a block are addressed with 32-bit vector offsets
+    if (int64_t(q.sc.n[s]) * (D / 8) >= INT32_MAX) return VARK_E_SHAPE;
+  if (layer_stride < int64_t(B) * H * q.sc.T * D) return VARK_E_ARG;
+  if (layer_stride % 8 != 0) return VARK_E_ALIGN;
   if (!aligned16(k) || !aligned16(v) || !aligned16(kq) || !aligned16(vq) || !aligned16(k_absmax) ||
       !aligned16(v_absmax))
     return VARK_E_ALIGN;
@@ -550,26 +791,32 @@ extern "C" int vark_quantize_kv_int8(const uint16_t* k, const uint16_t* v, int64
   if (cudaMemsetAsync(k_absmax, 0, size_t(nabs) * 4, st) != cudaSuccess ||
       cudaMemsetAsync(v_absmax, 0, size_t(nabs) * 4, st) != cudaSuccess)
     return VARK_E_CUDA;
-  p.L = L; p.B = B; p.H = H; p.D = D; p.layer_stride = layer_stride; p.src_rows = p.sc.T;
-  p.src_head_off = nullptr; p.src_seg_off = nullptr; p.src_layer_base = nullptr;
-  for (int s = 0; s < VARK_MAX_SCALES; ++s) {
-    p.chunks[s] = s < S ? (p.sc.n[s] + kChunkRows - 1) / kChunkRows : 0;
-    p.src_off[s] = s < S ? p.sc.off[s] : 0;
-  }
-  q.scale_stride_l = int64_t(B) * H * S * D;
+  q.L = L; q.B = B; q.H = H; q.D = D; q.layer_stride = layer_stride;
+  q.big_mask = 0;
+  for (int s = 0; s < S; ++s)
+    if (q.sc.n[s] > kSmallRows) q.big_mask |= 1u << s;
+  // as many clusters as can be resident at once (the unit loop is static)
   int dev = 0, nsm = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  const int layers_per_group = std::max(1, kMaxGroupLH / H);
-  for (int mode = 0; mode < 2; ++mode) {
-    q.mode = mode;
-    for (int l0 = 0; l0 < L; l0 += layers_per_group) {
-      p.l0 = l0;
-      p.nl = std::min(layers_per_group, L - l0);
-      quant_kernel<<<nsm * 4, kQuantThreads, 0, st>>>(k, v, q, keep, head_off, seg_off, layer_base, kq, vq,
-                                                      k_absmax, v_absmax);
-      if (cudaGetLastError() != cudaSuccess) return VARK_E_CUDA;
-    }
+  int clusters = 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(nsm * 4 / kQuantCluster * kQuantCluster);
+  cfg.blockDim = dim3(kQuantThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  if (cudaOccupancyMaxActiveClusters(&clusters, quant_kernel, &cfg) != cudaSuccess || clusters < 1) {
+    cudaGetLastError();
+    clusters = std::max(1, nsm / kQuantCluster);
+  }
+  const int layers_per_group = std::max(1, kQuantGroupLH / H);
+  for (int l0 = 0; l0 < L; l0 += layers_per_group) {
+    q.l0 = l0;
+    q.nl = std::min(layers_per_group, L - l0);
+    quant_kernel<<<clusters * kQuantCluster, kQuantThreads, 0, st>>>(
+        reinterpret_cast<const uint4*>(k), reinterpret_cast<const uint4*>(v), q, keep, head_off, seg_off, layer_base,
+        kq, vq, k_absmax, v_absmax);
+    if (cudaGetLastError() != cudaSuccess) return VARK_E_CUDA;
   }
   return VARK_OK;
 }
@@ -582,17 +829,19 @@ extern "C" int vark_dequantize_layer_int8(const int8_t* kq, const int8_t* vq, co
   DequantParams p;
   int rc = make_scale_table(S, sides, &p.sc);
   if (rc) return rc;
-  if (B < 1 || H < 1 || D < 4 || D % 4 != 0 || D > 512 || kc_rows < 0 || kc_rows % B != 0) return VARK_E_SHAPE;
-  if (!aligned16(k_absmax) || !aligned16(v_absmax) || (reinterpret_cast<uintptr_t>(kq) & 3) ||
-      (reinterpret_cast<uintptr_t>(vq) & 3) || !aligned16(kc) || !aligned16(vc))
+  if (B < 1 || H < 1 || H > kDeqMaxH || D < 8 || D % 8 != 0 || D > 512 || kc_rows < 0 || kc_rows % B != 0)
+    return VARK_E_SHAPE;
+  if (!aligned16(k_absmax) || !aligned16(v_absmax) || (reinterpret_cast<uintptr_t>(kq) & 7) ||
+      (reinterpret_cast<uintptr_t>(vq) & 7) || !aligned16(kc) || !aligned16(vc))
     return VARK_E_ALIGN;
   if ((rc = check_device_sm100())) return rc;
   if (kc_rows == 0) return VARK_OK;
-  p.B = B; p.H = H; p.D = D; p.rows = kc_rows;
+  p.B = B; p.H = H; p.D = D; p.R = kc_rows / B;
   int dev = 0, nsm = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  dequant_kernel<<<nsm * 8, 256, 0, static_cast<cudaStream_t>(stream)>>>(kq, vq, k_absmax, v_absmax, p, head_off,
-                                                                          seg_off, kc, vc);
+  dequant_kernel<<<nsm * 3, kDeqThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const uint2*>(kq), reinterpret_cast<const uint2*>(vq), k_absmax, v_absmax, p, head_off,
+      seg_off, reinterpret_cast<uint4*>(kc), reinterpret_cast<uint4*>(vc));
   return cudaGetLastError() == cudaSuccess ? VARK_OK : VARK_E_CUDA;
 }

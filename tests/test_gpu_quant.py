@@ -83,3 +83,67 @@ def test_int8_cache_bit_exact_and_attention(sides, D):
                     o_ref = oracle.pruned_attention_rows(f64(qb[b, h, g.off[kk] + rows_s]), k_eff, v_eff, keep[l, h],
                                                          sides, kk, float(tau[h].item()))
                     assert np.abs(O[b, h, g.off[kk] + rows_s] - o_ref).max() <= 2e-2, (l, b, h, kk)
+
+
+def _expected_layer_bf16(q_ref, a_ref, keep_l, g, ho_l, so_l, lb_l, R_l, B, H, D):
+    """The oracle's dequantised compacted block of one layer, [B * R_l][D] bf16 bits."""
+    out = np.zeros((B * R_l, D), dtype=np.uint16)
+    for b in range(B):
+        for h in range(H):
+            for s in range(g.S):
+                if not keep_l[h, s]:
+                    continue
+                r0 = b * R_l + int(ho_l[h]) + int(so_l[h, s])
+                codes = q_ref[lb_l + r0 * D:lb_l + (r0 + g.n[s]) * D].reshape(g.n[s], D)
+                out[r0:r0 + g.n[s]] = oracle.dequantize_block(codes, a_ref[b, h, s])
+    return out
+
+
+@pytest.mark.parametrize("sides,D,L,B,H,mode", [
+    (synth.SIDES_TINY, 96, 2, 3, 5, "random"),          # 12 vectors per row: a ragged thread layout
+    (synth.SIDES_1024, 256, 1, 2, 2, "all"),            # every block, the 4096-row one split over the cluster
+    (synth.SIDES_1024, 128, 2, 1, 3, "sparse"),         # a layer with nothing kept, a head with nothing kept
+    (synth.SIDES_TINY, 64, 3, 1, 1024, "random"),       # several (layer, head) launch groups
+    (synth.SIDES_1024, 8, 1, 2, 4, "random"),           # one vector per row
+])
+def test_int8_codes_and_dequant_bit_exact_shapes(sides, D, L, B, H, mode):
+    g = oracle.ScaleGeometry(sides)
+    T, S = g.T, g.S
+    kb = synth.normal_bf16_bits(synth.derive_key(97, D, H), (L, B, H, T, D))
+    vb = synth.normal_bf16_bits(synth.derive_key(98, D, H), (L, B, H, T, D))
+    rng = np.random.default_rng(D * 7 + H)
+    if mode == "all":
+        keep = np.ones((L, H, S), dtype=np.uint8)
+    else:
+        keep = rng.integers(0, 2, size=(L, H, S)).astype(np.uint8)
+    if mode == "sparse":
+        keep[0] = 0
+        keep[1, 1] = 0
+        keep[1, 0, -1] = 1
+    tab = Tables(keep, sides, B, D)
+    kd, vd = dev_bf16(kb), dev_bf16(vb)
+    kq = torch.full((max(tab.total, 16),), 77, dtype=torch.int8, device="cuda")
+    vq = torch.full_like(kq, 77)
+    ka = torch.full((L, B, H, S, D), 5.0, dtype=torch.float32, device="cuda")
+    va = torch.full_like(ka, 5.0)
+    vark.vark_quantize_kv_int8(kd, vd, B * H * T * D, L, B, H, sides, D, tab.keep, tab.head_off, tab.seg_off,
+                               tab.layer_base, kq, vq, ka, va)
+    torch.cuda.synchronize()
+    ho, so, pl, lb = oracle.build_offsets(keep, sides, B, D)
+    kq_ref, vq_ref, ka_ref, va_ref = oracle.quantize_kv(kb, vb, keep, sides, ho, so, lb)
+    assert np.array_equal(kq.cpu().numpy()[:tab.total], kq_ref)
+    assert np.array_equal(vq.cpu().numpy()[:tab.total], vq_ref)
+    assert np.array_equal(ka.cpu().numpy(), ka_ref) and np.array_equal(va.cpu().numpy(), va_ref)
+    for l in range(L):
+        rows = tab.kc_rows(l)
+        base = tab.elem_base(l)
+        kc = torch.zeros(max(rows * D, 16), dtype=torch.bfloat16, device="cuda")
+        vc = torch.zeros_like(kc)
+        vark.vark_dequantize_layer_int8(kq[base:], vq[base:], ka[l], va[l], rows, B, H, sides, D, tab.head_off[l],
+                                        tab.seg_off[l], kc, vc)
+        torch.cuda.synchronize()
+        R_l = rows // B
+        ek = _expected_layer_bf16(kq_ref, ka_ref[l], keep[l], g, ho[l], so[l], int(lb[l]), R_l, B, H, D)
+        ev = _expected_layer_bf16(vq_ref, va_ref[l], keep[l], g, ho[l], so[l], int(lb[l]), R_l, B, H, D)
+        assert np.array_equal(bits_of(kc)[:rows * D].reshape(-1, D), ek), l
+        assert np.array_equal(bits_of(vc)[:rows * D].reshape(-1, D), ev), l
