@@ -6,7 +6,8 @@ for the pruned-inference workload (32 layers, 16 heads, head_dim 128, 1024^2
 scale list, batch 8, 10% budget, sinks 0-1):
 
   1. S-CAS calibration attention of every layer (16 calibration seeds folded
-     into the batch)                                     vark_scas_accumulate
+     into the batch); the attention output O is written, as the layer's
+     output in a calibration forward pass        vark_scas_accumulate
   2. S-CAS finalisation and the greedy keep schedule (host) vark_scas_finalize,
                                                            vark_build_schedule
   3. offset tables                                       vark_build_offsets
@@ -183,6 +184,7 @@ class Pipeline:
         self.tau = torch.from_numpy(np.stack(taus)).to(device)
         self.bias = torch.from_numpy(np.stack(biases)).to(device)
         self.mass = torch.zeros((L, H, S, S), dtype=torch.float32, device=device)
+        self.cout = torch.empty((Bc, H, T, D), dtype=torch.bfloat16, device=device)   # calibration O, per layer
         self.out = torch.empty_like(self.q)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
         self.keep = torch.empty((L, H, S), dtype=torch.uint8, device=device)
@@ -211,7 +213,7 @@ class Pipeline:
         self.mass.zero_()
         for l in range(L):
             vark.vark_scas_accumulate(self.cq[l], self.ck[l], self.cv[l], self.sides, self.tau[l], self.bias[l],
-                                      self.mass[l], None, self.status)
+                                      self.mass[l], self.cout, self.status)
         rec("calib")
         self.mass_host.copy_(self.mass, non_blocking=True)
         st.synchronize()
@@ -270,7 +272,7 @@ class Pipeline:
         for l in range(L):
             ms.wait_event(ev_cal[l])
             vark.vark_scas_accumulate(self.cq[l], self.ck[l], self.cv[l], self.sides, self.tau[l], self.bias[l],
-                                      self.mass[l], None, self.status)
+                                      self.mass[l], self.cout, self.status)
         self.mass_host.copy_(self.mass, non_blocking=True)
         ms.synchronize()
         scas = vark.vark_scas_finalize(self.mass_host.numpy())
@@ -774,8 +776,9 @@ def profile_case(case: str, reps: int):
     if case == "calib":
         q, k, v = (randn_bf16((4, H, T, D), 10 + i, dev) for i in range(3))
         mass = torch.zeros((H, S, S), dtype=torch.float32, device=dev)
+        o = torch.empty_like(q)
         for _ in range(reps):
-            vark.vark_scas_accumulate(q, k, v, sides, tau, bias, mass, None, st)
+            vark.vark_scas_accumulate(q, k, v, sides, tau, bias, mass, o, st)
     else:
         L = 1 if case == "pruned" else 4
         B = w.batch

@@ -475,35 +475,40 @@ __device__ __forceinline__ QScale make_qscale(float a) {
 __device__ __forceinline__ float lo_bf16(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float hi_bf16(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-__device__ __forceinline__ uint32_t pack4_s8(float r0, float r1, float r2, float r3) {
-  const uint32_t c0 = uint32_t(__float2int_rn(r0)), c1 = uint32_t(__float2int_rn(r1));
-  const uint32_t c2 = uint32_t(__float2int_rn(r2)), c3 = uint32_t(__float2int_rn(r3));
-  return __byte_perm(__byte_perm(c0, c1, 0x0040), __byte_perm(c2, c3, 0x0040), 0x5410);
+// Adding kRound = 1.5 * 2^23 rounds a float of magnitude below 2^22 to an
+// integer (round to nearest, ties to even: the sum's ulp is 1), and the sum's
+// low byte is then that integer's two's-complement byte.
+constexpr float kRound = 12582912.0f;
+
+__device__ __forceinline__ uint32_t pack4_low_bytes(float y0, float y1, float y2, float y3) {
+  return __byte_perm(__byte_perm(__float_as_uint(y0), __float_as_uint(y1), 0x0040),
+                     __byte_perm(__float_as_uint(y2), __float_as_uint(y3), 0x0040), 0x5410);
 }
 
 __device__ __forceinline__ uint2 codes8(const uint4& x, const float (&sc)[8], const float (&rc)[8], bool force) {
   const float v[8] = {lo_bf16(x.x), hi_bf16(x.x), lo_bf16(x.y), hi_bf16(x.y),
                       lo_bf16(x.z), hi_bf16(x.z), lo_bf16(x.w), hi_bf16(x.w)};
-  float r[8], d[8];   // d > 1/2: the product lies within |t| * 2^-20 of a half-integer
+  float y[8], d[8];   // y: kRound + rint(t); d > 1/2: t lies within |t| * 2^-20 of a half-integer
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
-    const float t = v[j] * rc[j];
-    r[j] = rintf(t);
-    d[j] = fmaf(fabsf(t), 0x1p-20f, fabsf(t - r[j]));
+    const float t = __fmul_rn(v[j], rc[j]);
+    y[j] = __fadd_rn(t, kRound);
+    const float e = __fsub_rn(t, __fsub_rn(y[j], kRound));   // t - rint(t), exact
+    d[j] = fmaf(fabsf(t), 0x1p-20f, fabsf(e));
   }
   const float dmax = fmaxf(fmaxf(fmaxf(d[0], d[1]), fmaxf(d[2], d[3])), fmaxf(fmaxf(d[4], d[5]), fmaxf(d[6], d[7])));
   if (force || dmax > 0.5f) {   // rare: decide the flagged elements by the exact quotient
 #pragma unroll
     for (int j = 0; j < 8; ++j)
-      if (force || d[j] > 0.5f) r[j] = sc[j] == 0.f ? 0.f : rintf(__fdiv_rn(v[j], sc[j]));
+      if (force || d[j] > 0.5f) y[j] = __fadd_rn(sc[j] == 0.f ? 0.f : __fdiv_rn(v[j], sc[j]), kRound);
   }
   uint2 o;
-  o.x = pack4_s8(r[0], r[1], r[2], r[3]);
-  o.y = pack4_s8(r[4], r[5], r[6], r[7]);
+  o.x = pack4_low_bytes(y[0], y[1], y[2], y[3]);
+  o.y = pack4_low_bytes(y[4], y[5], y[6], y[7]);
   return o;
 }
 
-__global__ void __cluster_dims__(kQuantCluster, 1, 1) __launch_bounds__(kQuantThreads, 6) quant_kernel(
+__global__ void __cluster_dims__(kQuantCluster, 1, 1) __launch_bounds__(kQuantThreads, 5) quant_kernel(
     const uint4* __restrict__ k, const uint4* __restrict__ v, QuantParams p, const uint8_t* __restrict__ keep,
     const int32_t* __restrict__ head_off, const int32_t* __restrict__ seg_off, const int64_t* __restrict__ layer_base,
     int8_t* __restrict__ kq, int8_t* __restrict__ vq, float* __restrict__ ka, float* __restrict__ va) {
