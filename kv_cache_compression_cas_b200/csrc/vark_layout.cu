@@ -703,13 +703,20 @@ __global__ void __launch_bounds__(kDeqThreads, 3) dequant_kernel(const uint2* __
   if (threadIdx.x >= nrg * cv_n) return;   // no block-wide barrier follows
   const int cv = threadIdx.x % cv_n;
   const int rg = threadIdx.x / cv_n;
+  // Code byte i of w as a float, on the integer and FMA pipes: with the sign
+  // bit flipped the byte is k + 128, placed as the low mantissa byte of
+  // 1.5 * 2^23 (bits 0x4B400000) it reads 1.5 * 2^23 + k + 128, and one exact
+  // subtraction leaves k.
   auto expand = [](uint2 w, const float (&sc)[8]) {
-    auto x = [](uint32_t u, int i) { return float(int8_t((u >> (8 * i)) & 0xFFu)); };
+    const uint2 wf = make_uint2(w.x ^ 0x80808080u, w.y ^ 0x80808080u);
+    auto x = [](uint32_t u, int i) {
+      return __fsub_rn(__uint_as_float(__byte_perm(u, 0x4B400000u, 0x7640u | uint32_t(i))), 12583040.0f);
+    };
     uint4 o;
-    o.x = pack_bf16x2(x(w.x, 0) * sc[0], x(w.x, 1) * sc[1]);
-    o.y = pack_bf16x2(x(w.x, 2) * sc[2], x(w.x, 3) * sc[3]);
-    o.z = pack_bf16x2(x(w.y, 0) * sc[4], x(w.y, 1) * sc[5]);
-    o.w = pack_bf16x2(x(w.y, 2) * sc[6], x(w.y, 3) * sc[7]);
+    o.x = pack_bf16x2(__fmul_rn(x(wf.x, 0), sc[0]), __fmul_rn(x(wf.x, 1), sc[1]));
+    o.y = pack_bf16x2(__fmul_rn(x(wf.x, 2), sc[2]), __fmul_rn(x(wf.x, 3), sc[3]));
+    o.z = pack_bf16x2(__fmul_rn(x(wf.y, 0), sc[4]), __fmul_rn(x(wf.y, 1), sc[5]));
+    o.w = pack_bf16x2(__fmul_rn(x(wf.y, 2), sc[6]), __fmul_rn(x(wf.y, 3), sc[7]));
     return o;
   };
   // units in memory order (batch, head, kept chunk)
