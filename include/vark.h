@@ -343,7 +343,7 @@ int vark_recompact_kv(const uint16_t* kc_old, const uint16_t* vc_old, const int3
  * vark_quantize_kv_int8 -- device.  Compaction with quantisation: like
  * vark_compact_kv, but writes int8 codes to kq / vq (layer_base[L] bytes each)
  * and the per-(block, channel) absmax to k_absmax / v_absmax.  Each kept block
- * is read from HBM once (blocks of more than 256 rows are split over the CTAs
+ * is read from HBM once (blocks of more than 1024 rows are split over the CTAs
  * of a thread-block cluster, which exchange their partial maxima); the code
  * pass re-reads the rows from L2.  k, v, kq, vq, k_absmax, v_absmax 16-byte
  * aligned; layer_stride a multiple of 8.  Non-finite inputs: a NaN in a block
