@@ -68,6 +68,41 @@ __global__ void __launch_bounds__(1024) offsets_kernel(const uint8_t* __restrict
 }
 
 // ---------------------------------------------------------------- compaction
+// Exclusive scan of a[0, n) in shared memory by the whole block (kThreads
+// threads, each owning a contiguous segment); a[n] receives the total.
+template <int kThreads, int kMaxN>
+__device__ __forceinline__ void block_exclusive_scan(int32_t* a, int n, int32_t* warp_tot) {
+  constexpr int kPer = (kMaxN + kThreads - 1) / kThreads;
+  const int seg0 = threadIdx.x * kPer;
+  int32_t my_total = 0;
+  for (int u = 0; u < kPer; ++u)
+    if (seg0 + u < n) my_total += a[seg0 + u];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int32_t incl = my_total;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  int32_t warp_base = 0, grand = 0;
+#pragma unroll
+  for (int w = 0; w < kThreads / 32; ++w) {
+    if (w < warp) warp_base += warp_tot[w];
+    grand += warp_tot[w];
+  }
+  int32_t run = warp_base + incl - my_total;
+  for (int u = 0; u < kPer; ++u)
+    if (seg0 + u < n) {
+      const int32_t c = a[seg0 + u];
+      a[seg0 + u] = run;
+      run += c;
+    }
+  if (threadIdx.x == 0) a[n] = grand;
+  __syncthreads();
+}
+
 constexpr int kChunkRows = 64;
 constexpr int kCompactThreads = 256;
 constexpr int kMaxGroupLH = 4096;   // (layer, head) pairs per launch group
@@ -114,37 +149,9 @@ __global__ void __launch_bounds__(kCompactThreads, 4) compact_kernel(
     chunk_prefix[i] = c;
   }
   __syncthreads();
-  // 2. in-place exclusive scan: each thread owns a contiguous segment
-  constexpr int kPer = (kMaxGroupLH + kCompactThreads - 1) / kCompactThreads;
-  const int seg0 = threadIdx.x * kPer;
-  int32_t my_total = 0;
-  for (int u = 0; u < kPer; ++u)
-    if (seg0 + u < nlh) my_total += chunk_prefix[seg0 + u];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int32_t incl = my_total;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  if (lane == 31) warp_tot[warp] = incl;
-  __syncthreads();
-  int32_t warp_base = 0, grand = 0;
-#pragma unroll
-  for (int w = 0; w < kCompactThreads / 32; ++w) {
-    if (w < warp) warp_base += warp_tot[w];
-    grand += warp_tot[w];
-  }
-  int32_t run = warp_base + incl - my_total;
-  for (int u = 0; u < kPer; ++u) {
-    if (seg0 + u < nlh) {
-      const int32_t c = chunk_prefix[seg0 + u];
-      chunk_prefix[seg0 + u] = run;
-      run += c;
-    }
-  }
-  if (threadIdx.x == 0) chunk_prefix[nlh] = grand;
-  __syncthreads();
+  // 2. in-place exclusive scan; chunk_prefix[nlh] = total kept chunks
+  block_exclusive_scan<kCompactThreads, kMaxGroupLH>(chunk_prefix, nlh, warp_tot);
+  const int32_t grand = chunk_prefix[nlh];
 
   const int64_t units = int64_t(grand) * p.B;
   const int vec_per_row = p.D / 8;  // 16-byte vectors per row
@@ -347,9 +354,8 @@ extern "C" int vark_recompact_kv(const uint16_t* kc_old, const uint16_t* vc_old,
 //
 // Quantisation reads every kept byte from HBM once.  A unit is one block of
 // one tensor (K or V).  A block of at most kSmallRows rows (256 KB at D = 128)
-// belongs to one CTA:
-// a strided pass takes the channel maxima, a second pass over the same rows
-// (still in L2) writes the codes.  A larger block is split over the
+// belongs to one CTA: a strided pass takes the channel maxima, a second pass
+// over the same rows (still in L2) writes the codes.  A larger block is split over the
 // kQuantCluster CTAs of a thread-block cluster: each CTA reduces its slice,
 // the CTAs exchange partial maxima through distributed shared memory, then
 // each writes the codes of its slice.  Channel maxima are taken on the bf16
@@ -371,41 +377,6 @@ struct QuantParams {
   int L, B, H, D;
   int64_t layer_stride;     // elements between source layers
 };
-
-// Exclusive scan of a[0, n) in shared memory by the whole block (kThreads
-// threads, each owning a contiguous segment); a[n] receives the total.
-template <int kThreads, int kMaxN>
-__device__ __forceinline__ void block_exclusive_scan(int32_t* a, int n, int32_t* warp_tot) {
-  constexpr int kPer = (kMaxN + kThreads - 1) / kThreads;
-  const int seg0 = threadIdx.x * kPer;
-  int32_t my_total = 0;
-  for (int u = 0; u < kPer; ++u)
-    if (seg0 + u < n) my_total += a[seg0 + u];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int32_t incl = my_total;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  if (lane == 31) warp_tot[warp] = incl;
-  __syncthreads();
-  int32_t warp_base = 0, grand = 0;
-#pragma unroll
-  for (int w = 0; w < kThreads / 32; ++w) {
-    if (w < warp) warp_base += warp_tot[w];
-    grand += warp_tot[w];
-  }
-  int32_t run = warp_base + incl - my_total;
-  for (int u = 0; u < kPer; ++u)
-    if (seg0 + u < n) {
-      const int32_t c = a[seg0 + u];
-      a[seg0 + u] = run;
-      run += c;
-    }
-  if (threadIdx.x == 0) a[n] = grand;
-  __syncthreads();
-}
 
 struct QBlock {
   int l, h, s, b, t;        // t: 0 = K, 1 = V
@@ -452,7 +423,7 @@ __device__ __forceinline__ void absmax8(uint32_t (&acc)[4], const uint4& x) {
 }
 
 // Channel scale: sc = a / 127 (IEEE), and rc = RN(1 / sc) when the product
-// path is usable (sc normal and not tiny), else 0 (always divide).
+// path is usable (2^-100 <= sc <= 2^100), else 0 (always divide).
 struct QScale {
   float sc, rc;
 };
