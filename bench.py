@@ -463,6 +463,38 @@ def int8_cache(pipe, max_over_ranks, bf16_attention_ms, hbm_gbs, reps=3):
             "bf16_cache_attention_ms": bf16_attention_ms}
 
 
+def scas_only(pipe, max_over_ranks, with_o_ms, peaks, reps=2):
+    """Calibration of every layer called without an output buffer (S-CAS
+    only: the kernel skips V and the PV MMAs), timed with CUDA events outside
+    the step.  Algorithmic work here is the QK^T half of the calibration
+    FLOPs."""
+    import torch
+    vark, w = pipe.vark, pipe.w
+    st = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def run():
+        pipe.mass.zero_()
+        for l in range(w.layers):
+            vark.vark_scas_accumulate(pipe.cq[l], pipe.ck[l], pipe.cv[l], pipe.sides, pipe.tau[l], pipe.bias[l],
+                                      pipe.mass[l], None, pipe.status)
+    run()
+    torch.cuda.synchronize()
+    t = 0.0
+    for _ in range(reps):
+        e0.record(st)
+        run()
+        e1.record(st)
+        torch.cuda.synchronize()
+        t += e0.elapsed_time(e1) / 1e3
+    assert int(pipe.status.item()) == 0
+    t = max_over_ranks(t / reps)
+    qk = pipe.calib_flops / 2
+    return {"ms_per_step": t * 1e3, "with_output_ms_per_step": with_o_ms, "speedup": with_o_ms / (t * 1e3),
+            "qk_tflops": qk / t / 1e12, "qk_frac_of_bf16_peak": qk / t / 1e12 / peaks["bf16_tflops_sustained"],
+            "note": "all 32 layers, 16 seeds each; FLOPs = the QK^T half of the calibration work"}
+
+
 def ranking_stability(pipe):
     """S-CAS of every layer from two disjoint halves of the calibration seeds,
     compared by vark_rank_stability (Spearman over candidate pairs, Jaccard of
@@ -837,6 +869,7 @@ def main():
     ap.add_argument("--stability", type=int, default=1)
     ap.add_argument("--quant", type=int, default=1)
     ap.add_argument("--other-configs", type=int, default=1)
+    ap.add_argument("--scas-only", type=int, default=1)
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -972,6 +1005,9 @@ def main():
                "overlap": "per-layer H2D on a copy stream, D2H on a second stream, kernels wait on per-layer events"}
         del host_in, host_out
 
+    # ------------------------------------------------ S-CAS without the attention output
+    scas_o = scas_only(pipe, max_over_ranks, ph["calib"] * 1e3 / K, peaks) if args.scas_only else None
+
     # ------------------------------------------------ ranking stability (two disjoint seed halves)
     stab = ranking_stability(pipe) if args.stability else None
 
@@ -1020,7 +1056,7 @@ def main():
                                     "S-CAS, schedule, offsets, compaction, pruned attention of all layers"},
             "pruned_attention_tflops": pruned_tflops, "query_tokens_per_s": qtok_s, "compaction_gbs": comp_gbs,
             "roofline": roof, "kernels": kernels, "generation_order": gen, "ranking_stability": stab,
-            "int8_cache": quant, "other_configs": others,
+            "int8_cache": quant, "other_configs": others, "scas_without_output": scas_o,
             "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches,
             "clocks": clk, "peaks": peaks,

@@ -102,7 +102,9 @@ int vark_version(void);
  *   bias       dev  fp32 [H][S] additive logit bias per source scale, or NULL.
  *   mass       dev  fp32 [H][S][S], indexed [h][s][k]; accumulated with fp32
  *              atomics (one per (h, s, k) per CTA): entries s > k untouched.
- *   out        dev  bf16 [B][H][T][D] attention output O, or NULL to skip it.
+ *   out        dev  bf16 [B][H][T][D] attention output O, or NULL to skip it:
+ *              then v is not read and no PV product is formed (S-CAS only;
+ *              the mass is the same up to fp32 summation order).
  *   dev_status dev  int32, required; the caller sets it to 0 before the call;
  *              a kernel that gives up a bounded wait stores VARK_E_TIMEOUT.
  * Errors: VARK_E_ARG, VARK_E_SHAPE, VARK_E_ALIGN, VARK_E_CUDA, VARK_E_DEVICE.

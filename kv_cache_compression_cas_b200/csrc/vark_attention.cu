@@ -260,7 +260,10 @@ __device__ __forceinline__ int column_scale(const Params& p, const Item<PRUNED>&
   return it.k;
 }
 
-template <int D, bool PRUNED, bool MASS>
+// WITH_O = false (calibration called without an output): no V tiles and no PV
+// MMAs; the softmax releases S_X as soon as it has read it into registers, so
+// the next S MMA of that tile overlaps the rest of its softmax.
+template <int D, bool PRUNED, bool MASS, bool WITH_O>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kc,
@@ -325,6 +328,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         if (t.src == 0) tma_load_3d(dst, &tm_k, bar(kBarKFull + j), c * 64, t.row, it.bh);
         else tma_load_2d(dst, &tm_kc, bar(kBarKFull + j), c * 64, t.row);
       }
+      if (!WITH_O) continue;
       mbar_arrive_expect_tx(bar(kBarVFull + j), kTileBytes);
       for (int c = 0; c < QP; ++c) {
         const uint32_t dst = sV + j * kTileBytes + c * kPanelBytes;
@@ -349,7 +353,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       // (Q and the first kStages key tiles were issued right after the
       // barrier initialisation, by this same thread.)
       int issued_k = min(min(n, kStages), p.withhold_tile < 0 ? n : p.withhold_tile);
-      int issued_v = issued_k;
+      int issued_v = WITH_O ? issued_k : 0;
       for (int j = issued_k; j < n; ++j) {
         const int st = j % kStages;
         const KTile t = it.tile(p, j);
@@ -362,6 +366,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           else tma_load_2d(dst, &tm_kc, bar(kBarKFull + st), c * 64, t.row);
         }
         issued_k = j + 1;
+        if (!WITH_O) continue;
         if (j >= kStages && !mbar_wait(bar(kBarVEmpty + st), ((j / kStages) - 1) & 1, abort_flag, p.status, p.wait_limit_ns)) break;
         mbar_arrive_expect_tx(bar(kBarVFull + st), kTileBytes);
         for (int c = 0; c < QP; ++c) {
@@ -400,7 +405,22 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
       };
       bool ok = mbar_wait(bar(kBarQ), 0, abort_flag, p.status, p.wait_limit_ns);
-      for (int j = 0; ok && j < n; ++j) {
+      if (!WITH_O) {
+        // S MMAs only: S_X(j) once the softmax has read S_X(j-1)
+        for (int j = 0; ok && j < n; ++j) {
+          const int st = j % kStages;
+          if (!(ok = mbar_wait(bar(kBarKFull + st), (j / kStages) & 1, abort_flag, p.status, p.wait_limit_ns))) break;
+          for (int x = 0; x < n_act; ++x) {
+            if (j > 0 && !(ok = mbar_wait(bar(kBarPFull + x), (j - 1) & 1, abort_flag, p.status, p.wait_limit_ns))) break;
+            tc_fence_after();
+            issue_s(x, st);
+            mma_commit(bar(kBarSFull + x));
+          }
+          if (!ok) break;
+          if (j + kStages < n) mma_commit(bar(kBarKEmpty + st));
+        }
+      }
+      for (int j = 0; WITH_O && ok && j < n; ++j) {
         const int st = j % kStages, pst = (j + kStages - 1) % kStages;
         if (!(ok = mbar_wait(bar(kBarKFull + st), (j / kStages) & 1, abort_flag, p.status, p.wait_limit_ns))) break;
         if (j > 0 && !(ok = mbar_wait(bar(kBarVFull + pst), ((j - 1) / kStages) & 1, abort_flag, p.status, p.wait_limit_ns))) break;
@@ -419,7 +439,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         if (j + kStages < n) mma_commit(bar(kBarKEmpty + st));
         if (j > 0 && (j - 1) + kStages < n) mma_commit(bar(kBarVEmpty + pst));
       }
-      if (ok && n > 0) {
+      if (WITH_O && ok && n > 0) {
         const int pst = (n - 1) % kStages;
         ok = mbar_wait(bar(kBarVFull + pst), ((n - 1) / kStages) & 1, abort_flag, p.status, p.wait_limit_ns);
         for (int x = 0; ok && x < n_act; ++x) {
@@ -488,6 +508,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(v[c][i]);
         }
       }
+      if (!WITH_O) {   // S_X is in registers: the next S MMA of this tile may overwrite it
+        tc_fence_before();
+        mbar_arrive(bar(kBarPFull + x));
+      }
       float m_tile, sh;
       if (fast) {
         // one source scale, all columns valid: exponent = sv * qk2 + (b2 - m)
@@ -541,7 +565,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         if (MASS)
           for (int s = 0; s <= it.k; ++s) mrow[s * kBlockM] *= f;
       }
-      if (j > 0 && __any_sync(0xffffffffu, f != 1.f)) {
+      if (WITH_O && j > 0 && __any_sync(0xffffffffu, f != 1.f)) {
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t v[32];
@@ -606,7 +630,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
       }
       // P_X (bf16 pairs) over the first 64 columns of S_X
-      {
+      if (WITH_O) {
         uint32_t pk[2][32];
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
@@ -615,17 +639,17 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
         tmem_st32(tS, pk[0]);
         tmem_st32(tS + 32, pk[1]);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(kBarPFull + x));
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(kBarPFull + x));
     }
 
     // ---------------------------------------------------------- epilogue
-    if (ok && n > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarODone + x), 0, abort_flag, p.status, p.wait_limit_ns));
+    if (WITH_O && ok && n > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarODone + x), 0, abort_flag, p.status, p.wait_limit_ns));
     const bool row_ok = ok && r < it.rows_valid[x];
     const float inv_l = 1.f / l_sum;
-    if (ok && p.out != nullptr) {
+    if (WITH_O && ok && p.out != nullptr) {
       tc_fence_after();
       const int out_row = (p.q_scale_rows ? 0 : p.sc.off[it.k]) + it.row0 + x * kBlockM + r;
       uint16_t* orow = p.out + (int64_t(it.bh) * p.q_rows + out_row) * D;
@@ -733,11 +757,11 @@ static void apply_test_hooks(Params& p) {
   }
 }
 
-template <int D, bool PRUNED, bool MASS>
+template <int D, bool PRUNED, bool MASS, bool WITH_O = true>
 static int launch(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& kc,
                   const CUtensorMap& vc, Params& p, cudaStream_t st) {
   apply_test_hooks(p);
-  auto kern = attn_kernel<D, PRUNED, MASS>;
+  auto kern = attn_kernel<D, PRUNED, MASS, WITH_O>;
   const int smem = Smem<D>::alloc(MASS, p.sc.S);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
     cudaGetLastError();
@@ -781,6 +805,9 @@ extern "C" int vark_scas_accumulate(const uint16_t* q, const uint16_t* k, const 
   if ((rc = encode_dense(&tk, k, D, lp.sc.T, int64_t(B) * H))) return rc;
   if ((rc = encode_dense(&tv, v, D, lp.sc.T, int64_t(B) * H))) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (out == nullptr)   // S-CAS only: no V, no PV
+    return D == 128 ? launch<128, false, true, false>(tq, tk, tv, tk, tv, lp, st)
+                    : launch<64, false, true, false>(tq, tk, tv, tk, tv, lp, st);
   return D == 128 ? launch<128, false, true>(tq, tk, tv, tk, tv, lp, st)
                   : launch<64, false, true>(tq, tk, tv, tk, tv, lp, st);
 }

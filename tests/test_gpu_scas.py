@@ -94,6 +94,24 @@ def test_scas_1024_two_seeds_two_heads_full_parity():
     np.testing.assert_allclose(M_gpu, M_ref, rtol=MASS_RTOL, atol=MASS_ATOL)
 
 
+@pytest.mark.parametrize("sides,B,H,D", [(SIDES_TINY, 4, 4, 64), (SIDES_1024, 2, 2, 128), (SIDES_1024, 3, 1, 64)])
+def test_scas_without_output_matches_oracle(sides, B, H, D):
+    """S-CAS only (no output buffer): the kernel skips V and PV, and the mass
+    still matches the oracle and the with-output run."""
+    bits, tau, bias = _calib_inputs(sides, B, H, D, 7 + D, True)
+    M_noo, O_none = _gpu_calib(bits, sides, tau, bias, want_out=False)
+    assert O_none is None
+    M_o, _ = _gpu_calib(bits, sides, tau, bias, want_out=True)
+    q, k, v = (f64(b) for b in bits)
+    _, mass = oracle.block_causal_attention(q, k, v, sides, tau.astype(np.float64), bias.astype(np.float64))
+    M_ref = oracle.scas_mass(mass, sides)
+    np.testing.assert_allclose(M_noo, M_ref, rtol=MASS_RTOL, atol=MASS_ATOL)
+    np.testing.assert_allclose(M_noo, M_o, rtol=1e-5, atol=1e-7)
+    S = len(sides)
+    for kk in range(S):
+        np.testing.assert_allclose(M_noo[:, :kk + 1, kk].sum(axis=1), 1.0, atol=1e-4)
+
+
 @pytest.mark.slow
 def test_scas_calibration_full_size_sampled():
     """16 seeds x 16 heads at 1024^2, inputs made on the device: mass sums to
