@@ -951,7 +951,7 @@ def main():
     # dominant kernel: calibration attention (tensor-bound), timed inside a long step -> sustained peak
     per_launch_flops = w_calib / (K * L)
     per_launch_s = ph["calib"] / (K * L)
-    roof = {"bound": "tensor", "kernel": "attn_kernel<128,false,true> (S-CAS calibration attention)",
+    roof = {"bound": "tensor", "kernel": "attn_kernel<128,false,true,true> (S-CAS calibration attention, O written)",
             "achieved": per_launch_flops / per_launch_s / 1e12, "peak": peaks["bf16_tflops_sustained"],
             "unit": "TFLOP/s", "traffic": measured_traffic(),
             "traffic_source": "profiles/attn_calib_1024_4seeds_16heads.md (ncu dram bytes of a 4-seed launch x 4)",
