@@ -19,14 +19,14 @@ pytestmark = pytest.mark.gpu
 VARK_E_TIMEOUT = -6
 
 
-def _calib(sides, B, H, D, seed):
+def _calib(sides, B, H, D, seed, want_out=True):
     T = synth.n_tokens(sides)
     bits = [synth.normal_bf16_bits(synth.derive_key(90, seed, i), (B, H, T, D)) for i in range(3)]
     tau = synth.gen_tau(seed, H)
     q, k, v = (dev_bf16(b) for b in bits)
     S = len(sides)
     mass = torch.zeros((H, S, S), dtype=torch.float32, device="cuda")
-    out = torch.empty_like(q)
+    out = torch.empty_like(q) if want_out else None
     st = status_word()
     vark.vark_scas_accumulate(q, k, v, sides, torch.from_numpy(tau).cuda(), None, mass, out, st)
     torch.cuda.synchronize()
@@ -42,6 +42,9 @@ def test_withheld_key_tile_times_out_and_context_stays_usable(monkeypatch):
     dt = time.time() - t0
     assert status == VARK_E_TIMEOUT
     assert dt < 30.0
+    # S-CAS only (no output: no V, no PV) gives up the same way
+    status, *_ = _calib(sides, 1, 2, 128, 1, want_out=False)
+    assert status == VARK_E_TIMEOUT
     # pruned attention takes the same path
     B, H, D = 1, 2, 128
     T = synth.n_tokens(sides)
