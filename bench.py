@@ -316,6 +316,16 @@ class Pipeline:
         return {"calib_flops": self.calib_flops, "pruned_flops": pf, "comp_bytes": comp_bytes, "query_tokens": qtok}
 
 
+def arm_config(w, world):
+    """The `config` object of the JSON line (both arms)."""
+    return {"workload": WORKLOAD + ": 32 layers x 16 heads, head_dim 128, 1024^2 scales (10,521 tokens), "
+                                   "batch 8, budget 10%, sinks 0-1, calibration 16 seeds per layer",
+            "global_batch": w.batch * world, "seq_len": synth.n_tokens(w.sides),
+            "parallelism": f"replicas x{world}", "l2": "inputs larger than L2 (no flush needed)",
+            "value_def": "(calibration + pruned attention FLOPs) / step time; step = calibration, "
+                         "S-CAS, schedule, offsets, compaction, pruned attention of all layers"}
+
+
 def reference_arm(args, rank, world):
     """The oracle, as it stands, on the host cores: bounded samples of the
     workload per step."""
@@ -336,7 +346,7 @@ def reference_arm(args, rank, world):
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "sample": sample.describe()},
+            "config": arm_config(w, world),
             "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                              "sample": sample.describe()},
             "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -1048,12 +1058,7 @@ def main():
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": t_max * 1e3 / K, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": WORKLOAD + ": 32 layers x 16 heads, head_dim 128, 1024^2 scales (10,521 tokens), "
-                                   "batch 8, budget 10%, sinks 0-1, calibration 16 seeds per layer",
-                       "global_batch": w.batch * world, "seq_len": synth.n_tokens(w.sides),
-                       "parallelism": f"replicas x{world}", "l2": "inputs larger than L2 (no flush needed)",
-                       "value_def": "(calibration + pruned attention FLOPs) / step time; step = calibration, "
-                                    "S-CAS, schedule, offsets, compaction, pruned attention of all layers"},
+            "config": arm_config(w, world),
             "pruned_attention_tflops": pruned_tflops, "query_tokens_per_s": qtok_s, "compaction_gbs": comp_gbs,
             "roofline": roof, "kernels": kernels, "generation_order": gen, "ranking_stability": stab,
             "int8_cache": quant, "other_configs": others, "scas_without_output": scas_o,
