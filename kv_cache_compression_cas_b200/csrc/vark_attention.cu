@@ -63,6 +63,10 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 domain
 // is bound by instruction issue, not MUFU: shares of 2, 4, 6 per 8 ran 5-17%
 // slower than 0, so the polynomial path is off.
 constexpr int kPolyPer8 = 0;
+// Without an output (S-CAS only) there is no P -> PV -> S chain and the
+// softmax is bound by MUFU throughput: there 2 of 8 columns on the polynomial
+// measured 12% faster than 0 (4 of 8: 7%).
+constexpr int kPolyPer8NoO = 2;
 
 struct Params {
   ScaleTable sc;
@@ -584,10 +588,11 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         for (int c = 0; c < kBlockN; c += 2) ffma2(sv[c], sv[c + 1], sv[c], sv[c + 1], qk2, qk2, shm, shm);
 #pragma unroll
         for (int c = 0; c < kBlockN; c += 8) {
+          constexpr int kPoly = WITH_O ? kPolyPer8 : kPolyPer8NoO;
 #pragma unroll
-          for (int i = 0; i < kPolyPer8; i += 2) exp2_poly2(sv[c + i], sv[c + i + 1]);
+          for (int i = 0; i < kPoly; i += 2) exp2_poly2(sv[c + i], sv[c + i + 1]);
 #pragma unroll
-          for (int i = kPolyPer8; i < 8; ++i) sv[c + i] = ex2_approx(sv[c + i]);
+          for (int i = kPoly; i < 8; ++i) sv[c + i] = ex2_approx(sv[c + i]);
         }
       } else {
         const float shm = -m_used;
