@@ -124,3 +124,31 @@ def test_early_pruning_schedule_matches_oracle(sides, L, H, budget):
     p_ref, e_ref = oracle.early_pruning_schedule(scas, sides, budget, 2)
     p_got, e_got = vark.vark_build_early_pruning_schedule(scas, sides, budget, 2)
     assert np.array_equal(p_got, p_ref) and np.array_equal(e_got, e_ref)
+
+
+def test_generation_and_int8_calls_reject_bad_arguments_before_the_device():
+    lib = vark.library()
+    sides = (ctypes.c_int32 * 7)(*SIDES_TINY)
+    p = ctypes.c_void_p(16)
+    odd = ctypes.c_void_p(24)          # 8-byte but not 16-byte aligned
+    # quantising compaction: k, v, layer_stride, L, B, H, S, D, sides, keep, head_off, seg_off, layer_base, kq, vq, ka, va
+    assert lib.vark_quantize_kv_int8(None, p, 1 << 20, 1, 1, 4, 7, 64, sides, p, p, p, p, p, p, p, p, None) == -1
+    assert lib.vark_quantize_kv_int8(p, p, 1 << 20, 1, 1, 4, 7, 60, sides, p, p, p, p, p, p, p, p, None) == -2
+    assert lib.vark_quantize_kv_int8(p, p, 1 << 20, 1, 1, 4, 7, 1024, sides, p, p, p, p, p, p, p, p, None) == -2
+    assert lib.vark_quantize_kv_int8(p, p, 1 << 20, 1, 1, 4096, 7, 64, sides, p, p, p, p, p, p, p, p, None) == -2
+    assert lib.vark_quantize_kv_int8(p, p, 100, 1, 1, 4, 7, 64, sides, p, p, p, p, p, p, p, p, None) == -1
+    assert lib.vark_quantize_kv_int8(p, p, (1 << 20) + 4, 1, 1, 4, 7, 64, sides, p, p, p, p, p, p, p, p, None) == -3
+    assert lib.vark_quantize_kv_int8(p, p, 1 << 20, 1, 1, 4, 7, 64, sides, p, p, p, p, odd, p, p, p, None) == -3
+    # dequantisation: kq, vq, ka, va, kc_rows, B, H, S, D, sides, head_off, seg_off, kc, vc
+    assert lib.vark_dequantize_layer_int8(None, p, p, p, 8, 1, 4, 7, 64, sides, p, p, p, p, None) == -1
+    assert lib.vark_dequantize_layer_int8(p, p, p, p, 8, 1, 4, 7, 60, sides, p, p, p, p, None) == -2
+    assert lib.vark_dequantize_layer_int8(p, p, p, p, 9, 2, 4, 7, 64, sides, p, p, p, p, None) == -2
+    assert lib.vark_dequantize_layer_int8(p, p, p, p, 8, 1, 4, 7, 64, sides, p, p, odd, p, None) == -3
+    assert lib.vark_dequantize_layer_int8(ctypes.c_void_p(20), p, p, p, 8, 1, 4, 7, 64, sides, p, p, p, p,
+                                          None) == -3
+    # append of one scale: scale outside the list
+    assert lib.vark_append_scale(p, p, 1 << 20, 1, 1, 4, 7, 64, sides, 7, p, p, p, p, p, p, None) == -1
+    # re-compaction: the source and destination must differ; max_scale within [0, S]
+    assert lib.vark_recompact_kv(p, p, p, p, p, 1, 1, 4, 7, 64, sides, 3, p, p, p, p, p, p, None) == -1
+    q = ctypes.c_void_p(4096)
+    assert lib.vark_recompact_kv(p, p, p, p, p, 1, 1, 4, 7, 64, sides, 8, p, p, p, p, q, q, None) == -1
