@@ -35,12 +35,14 @@ from .layout import build_offsets, compact_kv
 from .generation import append_scale, cache_size_after_layer
 from .stability import rank_stability, average_ranks
 from .early_pruning import early_pruning_schedule, keep_after_step
-from .quant import quantize_block, dequantize_block, quantize_kv
+from .quant import (quantize_block, dequantize_block, quantize_kv, quantize_block_int4, dequantize_block_int4,
+                    pack_int4, unpack_int4, quantize_kv_int4, int4_scale_bits)
 
 __all__ = [
     "ScaleGeometry", "block_causal_attention", "attend", "scas_mass", "pruned_attention",
     "attention_rows", "pruned_attention_rows", "scas_from_mass", "build_schedule", "BudgetError", "full_cache_tokens",
     "build_offsets", "compact_kv", "append_scale", "cache_size_after_layer",
     "rank_stability", "average_ranks", "early_pruning_schedule", "keep_after_step",
-    "quantize_block", "dequantize_block", "quantize_kv",
+    "quantize_block", "dequantize_block", "quantize_kv", "quantize_block_int4", "dequantize_block_int4",
+    "pack_int4", "unpack_int4", "quantize_kv_int4", "int4_scale_bits",
 ]

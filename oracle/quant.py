@@ -74,3 +74,104 @@ def quantize_kv(k_dense, v_dense, keep, sides, head_off, seg_off, layer_base):
                     vq[dst:dst + geom.n[s] * D] = cv.ravel()
                     ka[l, b, h, s], va[l, b, h, s] = ak, av
     return kq, vq, ka, va
+
+
+# ---------------------------------------------------------------- 4-bit codes
+#
+# [VAR-Q] summary page: INT4 codes with (block, channel) groups match BF16
+# quality, and bit packing turns the nominal bit width into real memory
+# savings.  This library's 4-bit reading, on the same groups (a block is one
+# retained scale of one (layer, batch, head), one group per channel d):
+#
+#   a    = max |x| over the group (exact, from bf16 inputs)
+#   s    = bf16(a / 7)                 fp32 IEEE division, rounded to bf16 (RNE)
+#   code = clamp(rint(x / s), -7, 7)   fp32 IEEE division, round half to even;
+#                                      s = 0 gives 0
+#   x'   = bf16(code * s)              the product is exact in fp32 (at most 11
+#                                      significant bits), rounded once to bf16
+#
+# Storage: nibble = code + 8 (1..15); every 8 consecutive channels c0..c7 of a
+# row form one little-endian 32-bit word with the even channels c0, c2, c4, c6
+# in nibbles 0-3 and the odd channels c1, c3, c5, c7 in nibbles 4-7, so a row
+# of D channels is D/2 bytes.  Scales are kept as bf16 bits.
+#
+# Parity: exact arithmetic on both sides (bit-exact codes, scales, packed
+# bytes, dequantised bf16); pinned by the error bound |x' - x| <= s/2 +
+# |x'| 2^-9, exactness on the integer grid, the absmax element mapping to +-7,
+# zero blocks, a hand-packed word, and identity-coded placement.
+
+def int4_scale_bits(a):
+    """bf16 bits of s = bf16(a / 7) for fp32 absmax values a."""
+    return _bf16((np.asarray(a, dtype=np.float32) / np.float32(7.0)).astype(np.float32))
+
+
+def quantize_block_int4(x_bits):
+    """x_bits: uint16 bf16 [rows][D].  Returns (codes int8 [rows][D] in
+    [-7, 7], scale bf16 bits uint16 [D])."""
+    x = _f32(x_bits)
+    a = np.abs(x).max(axis=0).astype(np.float32)
+    s_bits = int4_scale_bits(a)
+    s = _f32(s_bits)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        t = np.rint((x / s[None, :]).astype(np.float32))
+    t = np.where(s[None, :] == 0, 0, t)
+    return np.clip(t, -7, 7).astype(np.int8), s_bits
+
+
+def dequantize_block_int4(codes, s_bits):
+    s = _f32(s_bits)
+    return _bf16((np.asarray(codes).astype(np.float32) * s[None, :]).astype(np.float32))
+
+
+def pack_int4(codes):
+    """int8 [rows][D] (D % 8 == 0) -> uint8 [rows][D/2] in the nibble layout above."""
+    codes = np.asarray(codes)
+    rows, D = codes.shape
+    nib = (codes.astype(np.int64) + 8).astype(np.uint32).reshape(rows, D // 8, 8)
+    word = np.zeros((rows, D // 8), dtype=np.uint32)
+    for j in range(4):
+        word |= nib[:, :, 2 * j] << np.uint32(4 * j)
+        word |= nib[:, :, 2 * j + 1] << np.uint32(16 + 4 * j)
+    return word.astype("<u4").view(np.uint8).reshape(rows, D // 2)
+
+
+def unpack_int4(packed, D):
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    rows = packed.size // (D // 2)
+    word = packed.reshape(rows, D // 2).view("<u4").astype(np.uint32)
+    codes = np.zeros((rows, D // 8, 8), dtype=np.int64)
+    for j in range(4):
+        codes[:, :, 2 * j] = ((word >> np.uint32(4 * j)) & 0xF).astype(np.int64) - 8
+        codes[:, :, 2 * j + 1] = ((word >> np.uint32(16 + 4 * j)) & 0xF).astype(np.int64) - 8
+    return codes.reshape(rows, D).astype(np.int8)
+
+
+def quantize_kv_int4(k_dense, v_dense, keep, sides, head_off, seg_off, layer_base):
+    """Dense uint16 [L][B][H][T][D] -> (kq, vq uint8 packed, layer_base[L] / 2
+    bytes each; k_scale, v_scale bf16 bits uint16 [L][B][H][S][D], 0 for
+    dropped scales).  Element e of the compacted layout has its nibble in
+    byte e / 2 of the packed buffer (rows of D / 2 bytes)."""
+    keep = np.asarray(keep)
+    L, B, H, T, D = k_dense.shape
+    geom = ScaleGeometry(sides)
+    total = int(layer_base[L])
+    kq = np.zeros(total // 2, dtype=np.uint8)
+    vq = np.zeros(total // 2, dtype=np.uint8)
+    ks = np.zeros((L, B, H, geom.S, D), dtype=np.uint16)
+    vs = np.zeros((L, B, H, geom.S, D), dtype=np.uint16)
+    for l in range(L):
+        R_l = int(layer_base[l + 1] - layer_base[l]) // (B * D)
+        for b in range(B):
+            for h in range(H):
+                for s in range(geom.S):
+                    if not keep[l, h, s]:
+                        continue
+                    sl = slice(geom.off[s], geom.off[s] + geom.n[s])
+                    ck, sk = quantize_block_int4(k_dense[l, b, h, sl])
+                    cv, sv = quantize_block_int4(v_dense[l, b, h, sl])
+                    row = b * R_l + int(head_off[l, h]) + int(seg_off[l, h, s])
+                    dst = (int(layer_base[l]) + row * D) // 2
+                    kq[dst:dst + geom.n[s] * D // 2] = pack_int4(ck).ravel()
+                    vq[dst:dst + geom.n[s] * D // 2] = pack_int4(cv).ravel()
+                    ks[l, b, h, s], vs[l, b, h, s] = sk, sv
+    return kq, vq, ks, vs
