@@ -60,22 +60,32 @@ def _peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-def measured_traffic():
-    """DRAM bytes per full calibration launch from the committed ncu summary,
-    or None when the attention kernel's source has changed since the capture."""
+TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "traffic.json")
+ATTN_SOURCES = [os.path.join(ROOT, "kv_cache_compression_cas_b200", "csrc", f)
+                for f in ("vark_attention.cu", "vark_common.cuh")]
+
+
+def attention_source_hash():
     import hashlib
-    import re
-    prof = os.path.join(ROOT, "profiles", "attn_calib_1024_4seeds_16heads.md")
-    src = os.path.join(ROOT, "kv_cache_compression_cas_b200", "csrc", "vark_attention.cu")
+    h = hashlib.sha256()
+    for f in ATTN_SOURCES:
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic():
+    """(DRAM bytes per full calibration launch, capture note) from the
+    committed capture record, or (None, reason) when the attention kernel's
+    source has changed since the capture."""
     try:
-        text = open(prof).read()
-        m = re.search(r"Traffic per full launch \(bytes\): (\d+) \(kernel ([0-9a-f]+)\)", text)
-        cur = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    except OSError:
-        return None
-    if not m or m.group(2) != cur:
-        return None
-    return int(m.group(1))
+        with open(TRAFFIC_RECORD) as f:
+            rec = json.load(f)["attn_kernel<128,false,true,true>"]
+    except (OSError, KeyError, ValueError):
+        return None, "no capture record"
+    if rec.get("source_sha16") != attention_source_hash():
+        return None, "kernel changed since the capture"
+    return int(rec["dram_bytes_per_launch"]), rec.get("capture", "")
 
 
 # ---------------------------------------------------------------- algorithmic work
@@ -157,6 +167,12 @@ def randn_bf16(shape, seed, device):
     return t
 
 
+def replica_seed(w: synth.Workload, rank: int) -> int:
+    """Seed of one rank's replica: every rank draws its own inputs (weak
+    scaling over independent replicas, no data-path exchange)."""
+    return synth.derive_key(w.base_seed, 0xBE, rank)
+
+
 # ---------------------------------------------------------------- the pipeline
 class Pipeline:
     """Device buffers and one step of the hot path for one rank."""
@@ -171,7 +187,7 @@ class Pipeline:
         self.T = synth.n_tokens(w.sides)
         L, B, H, D, T, S = w.layers, w.batch, w.heads, w.head_dim, self.T, self.S
         Bc = w.n_seeds
-        seed = synth.derive_key(w.base_seed, 0xBE, rank)
+        seed = replica_seed(w, rank)
         # calibration inputs: per layer [seeds][H][T][D]; inference: [L][B][H][T][D]
         self.cq = randn_bf16((L, Bc, H, T, D), seed + 1, device)
         self.ck = randn_bf16((L, Bc, H, T, D), seed + 2, device)
@@ -348,18 +364,26 @@ def reference_arm(args, rank, world):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": arm_config(w, world),
             "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                             "sample": sample.describe()},
+                             "sample": sample.describe(), "per_step": sample.per_step()},
             "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
 
 
 class CpuSample:
-    """A bounded slice of one step for the oracle: calibration attention of
-    one seed and one head of one layer, the S-CAS finalisation and schedule of
-    all 32 layers, the offsets of all layers, the compaction of one (layer,
-    batch) element and the pruned attention of two heads of one batch
-    element of one layer.  Work is counted in algorithmic attention FLOPs."""
+    """A bounded slice of one step for the oracle, each part timed on its own
+    and reported in the GPU path's unit for that part:
+
+    * calibration attention of one seed and one head of one layer at full T
+      (TFLOP/s);
+    * S-CAS finalisation + schedule of all 32 layers (in full, ms);
+    * offsets of all 32 layers (in full, ms);
+    * compaction of one (layer, batch) element (GB/s, read + write);
+    * pruned attention of two heads of one batch element of one layer
+      (TFLOP/s and query tokens/s).
+
+    Full-step seconds are extrapolated linearly from each slice by the
+    algorithmic work ratio and labelled so."""
 
     def __init__(self, w):
         import oracle
@@ -376,6 +400,9 @@ class CpuSample:
         self.tau = synth.gen_tau(key, H).astype(np.float64)
         self.bias = synth.gen_bias(key, H, S).astype(np.float64)
         self.M = np.random.default_rng(1).uniform(0, 1, size=(w.layers, H, S, S))
+        self.t = {k: 0.0 for k in ("calibration", "schedule", "offsets", "compaction", "pruned_attention")}
+        self.work = {k: 0.0 for k in self.t}
+        self.full = None
 
     def describe(self):
         return ("oracle fp64 slice per step: calibration attention of 1 seed x 1 head x 1 layer at full T, "
@@ -383,27 +410,82 @@ class CpuSample:
                 "1 batch x 2 heads x 1 layer; FLOPs counted as on the GPU")
 
     def run(self, small=False):
+        """One slice; returns its attention FLOPs (calibration + pruned)."""
         o, w, g = self.o, self.w, self.g
         D = w.head_dim
-        flops = 0.0
         q, k, v = self.qkv
-        heads = 1
-        o.block_causal_attention(q[:, :heads], k[:, :heads], v[:, :heads], self.sides, self.tau[:heads],
-                                 self.bias[:heads])
-        flops += calib_flops(self.sides, 1, heads, D)
+        tic = time.perf_counter()
+        o.block_causal_attention(q[:, :1], k[:, :1], v[:, :1], self.sides, self.tau[:1], self.bias[:1])
+        cf = calib_flops(self.sides, 1, 1, D)
         if small:
-            return flops
+            return cf
+        self.t["calibration"] += time.perf_counter() - tic
+        self.work["calibration"] += cf
+        tic = time.perf_counter()
         scas = o.scas_from_mass(self.M)
         keep = o.build_schedule(scas, self.sides, w.budget_bp, w.n_sinks)
-        ho, so, pl, lb = o.build_offsets(keep, self.sides, w.batch, D)
+        self.t["schedule"] += time.perf_counter() - tic
+        self.work["schedule"] += 1
+        tic = time.perf_counter()
+        o.build_offsets(keep, self.sides, w.batch, D)
+        self.t["offsets"] += time.perf_counter() - tic
+        self.work["offsets"] += 1
         k1 = keep[:1]
         ho1, so1, pl1, lb1 = o.build_offsets(k1, self.sides, 1, D)
+        tic = time.perf_counter()
         o.compact_kv(self.kbits, self.vbits, k1, self.sides, ho1, so1, lb1)
+        self.t["compaction"] += time.perf_counter() - tic
+        self.work["compaction"] += 2.0 * int(lb1[-1]) * 2 * 2          # read + write, K and V, bf16
         kd = (self.kbits[0].astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
         vd = (self.vbits[0].astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+        tic = time.perf_counter()
         o.pruned_attention(q[:, :2], kd[:, :2], vd[:, :2], keep[0, :2], self.sides, self.tau[:2], self.bias[:2])
-        flops += pruned_flops(keep[:1, :2], self.sides, 1, D)
-        return flops
+        self.t["pruned_attention"] += time.perf_counter() - tic
+        pf = pruned_flops(keep[:1, :2], self.sides, 1, D)
+        self.work["pruned_attention"] += pf
+        if self.full is None:
+            n = np.array([x * x for x in self.sides], dtype=np.int64)
+            kept = int((keep.astype(np.int64) * n[None, None, :]).sum())
+            self.full = {"calibration": calib_flops(self.sides, w.n_seeds, w.heads, D) * w.layers,
+                         "compaction": 2.0 * kept * w.batch * D * 2 * 2,
+                         "pruned_attention": pruned_flops(keep, self.sides, w.batch, D),
+                         "query_tokens": float(w.layers * w.batch * g.T)}
+        return cf + pf
+
+    def per_step(self):
+        """Each part's rate in the GPU path's unit, with the full-step seconds
+        extrapolated from the slice."""
+        t, wk, full = self.t, self.work, self.full
+        if not full or t["calibration"] <= 0:
+            return None
+        reps = wk["schedule"]
+        g = self.g
+        q_rows_slice = 2.0 * g.T                # 2 heads x all query rows of one batch element
+        out = {
+            "calibration_attention": {
+                "tflops": wk["calibration"] / t["calibration"] / 1e12,
+                "sample": "1 seed x 1 head x 1 layer, full T",
+                "full_step_s_extrapolated": full["calibration"] / (wk["calibration"] / t["calibration"]),
+                "scaling": "linear in algorithmic FLOPs (x%d)" % round(full["calibration"] / (wk["calibration"] / reps))},
+            "scas_finalise_and_schedule": {"ms": t["schedule"] / reps * 1e3, "sample": "all 32 layers (full)"},
+            "offsets": {"ms": t["offsets"] / reps * 1e3, "sample": "all 32 layers (full)"},
+            "compaction": {
+                "gbs": wk["compaction"] / t["compaction"] / 1e9,
+                "sample": "1 (layer, batch) element of the 32 x 8",
+                "full_step_s_extrapolated": full["compaction"] / (wk["compaction"] / t["compaction"]),
+                "scaling": "linear in bytes moved"},
+            "pruned_attention": {
+                "tflops": wk["pruned_attention"] / t["pruned_attention"] / 1e12,
+                "query_tokens_per_s": q_rows_slice * reps / t["pruned_attention"],
+                "sample": "1 batch element x 2 heads x 1 layer, all 13 query scales",
+                "full_step_s_extrapolated": full["pruned_attention"] / (wk["pruned_attention"] / t["pruned_attention"]),
+                "scaling": "linear in algorithmic FLOPs"},
+        }
+        out["full_step_s_extrapolated"] = (out["calibration_attention"]["full_step_s_extrapolated"]
+                                           + out["compaction"]["full_step_s_extrapolated"]
+                                           + out["pruned_attention"]["full_step_s_extrapolated"]
+                                           + (t["schedule"] + t["offsets"]) / reps)
+        return out
 
 
 def int8_cache(pipe, max_over_ranks, bf16_attention_ms, hbm_gbs, reps=3):
@@ -471,6 +553,70 @@ def int8_cache(pipe, max_over_ranks, bf16_attention_ms, hbm_gbs, reps=3):
             "dequantize_frac_of_hbm": q_bytes / td / 1e9 / hbm_gbs,
             "dequant_plus_attention_ms": ta * 1e3,
             "bf16_cache_attention_ms": bf16_attention_ms}
+
+
+def int4_cache(pipe, max_over_ranks, bf16_attention_ms, hbm_gbs, reps=3):
+    """The retained cache stored as packed 4-bit codes with per-(block,
+    channel) bf16 scales: quantising compaction of all layers, then per layer
+    dequantisation into a one-layer bf16 buffer followed by that layer's
+    pruned attention."""
+    import torch
+    vark, w = pipe.vark, pipe.w
+    L, B, H, D, S, T = w.layers, w.batch, w.heads, w.head_dim, pipe.S, pipe.T
+    base = pipe.base_host.numpy()
+    total = int(base[-1])
+    dev = pipe.dev
+    kq = torch.empty(max(total // 2, 16), dtype=torch.uint8, device=dev)
+    vq = torch.empty_like(kq)
+    ks = torch.empty((L, B, H, S, D), dtype=torch.int16, device=dev)
+    vs = torch.empty_like(ks)
+    max_rows = max(int(base[l + 1] - base[l]) // D for l in range(L))
+    kcl = torch.empty(max(max_rows * D, 16), dtype=torch.bfloat16, device=dev)
+    vcl = torch.empty_like(kcl)
+    st = torch.cuda.current_stream()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+
+    def one():
+        ev[0].record(st)
+        vark.vark_quantize_kv_int4(pipe.k, pipe.v, B * H * T * D, L, B, H, pipe.sides, D, pipe.keep, pipe.head_off,
+                                   pipe.seg_off, pipe.layer_base, kq, vq, ks, vs)
+        ev[1].record(st)
+        for l in range(L):
+            rows = int(base[l + 1] - base[l]) // D
+            b0 = int(base[l]) // 2
+            vark.vark_dequantize_layer_int4(kq[b0:], vq[b0:], ks[l], vs[l], rows, B, H, pipe.sides, D,
+                                            pipe.head_off[l], pipe.seg_off[l], kcl, vcl)
+            vark.vark_pruned_attention(pipe.q[l], kcl if rows else None, vcl if rows else None, rows, pipe.k[l],
+                                       pipe.v[l], pipe.sides, -1, pipe.head_off[l], pipe.seg_off[l],
+                                       pipe.past_len[l], pipe.tau[l], pipe.bias[l], pipe.out[l], pipe.status)
+        ev[2].record(st)
+        for l in range(L):     # the dequantisations alone
+            rows = int(base[l + 1] - base[l]) // D
+            b0 = int(base[l]) // 2
+            vark.vark_dequantize_layer_int4(kq[b0:], vq[b0:], ks[l], vs[l], rows, B, H, pipe.sides, D,
+                                            pipe.head_off[l], pipe.seg_off[l], kcl, vcl)
+        ev[3].record(st)
+
+    one()
+    torch.cuda.synchronize()
+    tq = ta = td = 0.0
+    for _ in range(reps):
+        one()
+        torch.cuda.synchronize()
+        tq += ev[0].elapsed_time(ev[1]) / 1e3
+        ta += ev[1].elapsed_time(ev[2]) / 1e3
+        td += ev[2].elapsed_time(ev[3]) / 1e3
+    assert int(pipe.status.item()) == 0
+    tq, ta, td = max_over_ranks(tq / reps), max_over_ranks(ta / reps), max_over_ranks(td / reps)
+    bf16_bytes = 2 * 2 * total
+    int4_bytes = 2 * (total // 2) + 2 * 2 * ks.numel()
+    q_bytes = bf16_bytes + int4_bytes     # kept bf16 K, V read once; packed codes and scale tables written
+    return {"cache_bytes_bf16": bf16_bytes, "cache_bytes_int4": int4_bytes, "cache_ratio": int4_bytes / bf16_bytes,
+            "quantize_ms": tq * 1e3, "quantize_gbs": q_bytes / tq / 1e9,
+            "quantize_frac_of_hbm": q_bytes / tq / 1e9 / hbm_gbs,
+            "dequantize_ms": td * 1e3, "dequantize_gbs": q_bytes / td / 1e9,
+            "dequantize_frac_of_hbm": q_bytes / td / 1e9 / hbm_gbs,
+            "dequant_plus_attention_ms": ta * 1e3, "bf16_cache_attention_ms": bf16_attention_ms}
 
 
 def scas_only(pipe, max_over_ranks, with_o_ms, peaks, reps=2):
@@ -787,6 +933,36 @@ def early_pruning_order(pipe, per_scale, outs, passes, max_over_ranks, sum_over_
             "bytes_moved_per_pass": moved}
 
 
+def summarize_kernels(kernels, quant, quant4, others, scas_o, peaks):
+    """Rounded per-kernel rates and roofline fractions (sustained / burst)."""
+    bs, bb, hb = peaks["bf16_tflops_sustained"], peaks["bf16_tflops"], peaks["hbm_gbs"]
+    r = lambda x: None if x is None else round(float(x), 3)
+    out = {"calibration_tflops": r(kernels["scas_calibration_attention"]["tflops"]),
+           "calibration_frac": [r(kernels["scas_calibration_attention"]["tflops"] / bs),
+                                r(kernels["scas_calibration_attention"]["tflops"] / bb)],
+           "pruned_tflops": r(kernels["pruned_attention"]["tflops"]),
+           "pruned_frac": [r(kernels["pruned_attention"]["tflops"] / bs), r(kernels["pruned_attention"]["tflops"] / bb)],
+           "pruned_query_tokens_per_s": r(kernels["pruned_attention"]["query_tokens_per_s"]),
+           "compaction_gbs": r(kernels["compaction"]["gbs"]), "compaction_frac_of_hbm": r(kernels["compaction"]["gbs"] / hb),
+           "fractions": "[of sustained, of burst] bf16 peak"}
+    if scas_o:
+        out["scas_only_qk_tflops"] = r(scas_o["qk_tflops"])
+    if quant:
+        out["int8"] = {"cache_ratio": r(quant["cache_ratio"]), "quantize_frac_of_hbm": r(quant["quantize_frac_of_hbm"]),
+                       "dequantize_frac_of_hbm": r(quant["dequantize_frac_of_hbm"])}
+    if quant4:
+        out["int4"] = {"cache_ratio": r(quant4["cache_ratio"]), "quantize_frac_of_hbm": r(quant4["quantize_frac_of_hbm"]),
+                       "dequantize_frac_of_hbm": r(quant4["dequantize_frac_of_hbm"]),
+                       "dequant_plus_attention_vs_bf16": r(quant4["dequant_plus_attention_ms"] / quant4["bf16_cache_attention_ms"])}
+    if others:
+        l8 = others["large_8l"]
+        out["large_8l"] = {"calibration_tflops": r(l8["calibration_tflops"]), "pruned_tflops": r(l8["pruned_attention_tflops"]),
+                           "compaction_gbs": r(l8["compaction_gbs"]), "compaction_frac_of_hbm": r(l8["compaction_frac_of_hbm"])}
+        out["final_scale_frac_of_burst"] = {f"B{p['batch']}_{p['budget_bp']}bp": r(p["frac_of_bf16_peak"])
+                                            for p in others["final_scale"]["points"]}
+    return out
+
+
 def reduce_over_ranks(x: float, op: str, world: int, device) -> float:
     """Max or sum of a host float over all ranks (timing plumbing; no data-path
     collective).  Works with NCCL (CUDA device) and gloo (CPU device)."""
@@ -802,10 +978,13 @@ def reduce_over_ranks(x: float, op: str, world: int, device) -> float:
 def profile_case(case: str, reps: int):
     """Small single-kernel runs for Nsight Compute captures (inputs > L2, a
     few GB at most): 'calib' = calibration attention, 4 seeds x 16 heads at
-    1024^2; 'pruned' = pruned attention of one layer of the 32-layer
+    1024^2; 'calib16' = one calibration launch exactly as the benchmark step
+    runs it (16 seeds x 16 heads, 2 GB of inputs; for single-pass DRAM
+    counters); 'pruned' = pruned attention of one layer of the 32-layer
     workload (batch 8, 10% budget schedule); 'compact' = compaction of 4
     layers of that workload; 'quant' = int8 quantising compaction of those 4
-    layers, then the dequantisation of each."""
+    layers, then the dequantisation of each; 'quant4' = 4-bit quantising
+    compaction of those 4 layers, then the dequantisation of each."""
     import torch
     import kv_cache_compression_cas_b200 as vark
     dev = torch.device("cuda", 0)
@@ -815,8 +994,9 @@ def profile_case(case: str, reps: int):
     st = torch.zeros(1, dtype=torch.int32, device=dev)
     tau = torch.from_numpy(synth.gen_tau(1, H)).to(dev)
     bias = torch.from_numpy(synth.gen_bias(1, H, S)).to(dev)
-    if case == "calib":
-        q, k, v = (randn_bf16((4, H, T, D), 10 + i, dev) for i in range(3))
+    if case in ("calib", "calib16"):
+        seeds = 4 if case == "calib" else w.n_seeds
+        q, k, v = (randn_bf16((seeds, H, T, D), 10 + i, dev) for i in range(3))
         mass = torch.zeros((H, S, S), dtype=torch.float32, device=dev)
         o = torch.empty_like(q)
         for _ in range(reps):
@@ -837,6 +1017,21 @@ def profile_case(case: str, reps: int):
         kc = torch.empty(max(total, 8), dtype=torch.bfloat16, device=dev)
         vc = torch.empty_like(kc)
         reps_c = reps if case == "compact" else 1
+        if case == "quant4":
+            kq4 = torch.empty(max(total // 2, 16), dtype=torch.uint8, device=dev)
+            vq4 = torch.empty_like(kq4)
+            ks4 = torch.empty((L, B, H, S, D), dtype=torch.int16, device=dev)
+            vs4 = torch.empty_like(ks4)
+            for _ in range(reps):
+                vark.vark_quantize_kv_int4(k, v, B * H * T * D, L, B, H, sides, D, keep_d, ho, so, lb, kq4, vq4, ks4,
+                                           vs4)
+            base4 = lb.cpu().numpy()
+            for _ in range(reps):
+                for l in range(L):
+                    rows = int(base4[l + 1] - base4[l]) // D
+                    vark.vark_dequantize_layer_int4(kq4[int(base4[l]) // 2:], vq4[int(base4[l]) // 2:], ks4[l], vs4[l],
+                                                    rows, B, H, sides, D, ho[l], so[l], kc, vc)
+            reps_c = 0
         for _ in range(reps_c):
             vark.vark_compact_kv(k, v, B * H * T * D, L, B, H, sides, D, keep_d, ho, so, lb, kc, vc)
         if case == "quant":
@@ -867,7 +1062,8 @@ def profile_case(case: str, reps: int):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--profile-case", choices=["calib", "pruned", "compact", "quant"], default=None)
+    ap.add_argument("--profile-case", choices=["calib", "calib16", "pruned", "compact", "quant", "quant4"],
+                    default=None)
     ap.add_argument("--profile-reps", type=int, default=3)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=5)
@@ -961,12 +1157,14 @@ def main():
     # dominant kernel: calibration attention (tensor-bound), timed inside a long step -> sustained peak
     per_launch_flops = w_calib / (K * L)
     per_launch_s = ph["calib"] / (K * L)
+    traffic, traffic_note = measured_traffic()
     roof = {"bound": "tensor", "kernel": "attn_kernel<128,false,true,true> (S-CAS calibration attention, O written)",
             "achieved": per_launch_flops / per_launch_s / 1e12, "peak": peaks["bf16_tflops_sustained"],
-            "unit": "TFLOP/s", "traffic": measured_traffic(),
-            "traffic_source": "profiles/attn_calib_1024_4seeds_16heads.md (ncu dram bytes of a 4-seed launch x 4)",
-            "peak_kind": f"bf16 dense sustained ({peaks['source']})"}
+            "unit": "TFLOP/s", "traffic": traffic, "traffic_source": "profiles/traffic.json: " + traffic_note,
+            "algorithmic_bytes_per_launch": 2.0 * 4 * w.n_seeds * w.heads * pipe.T * w.head_dim,
+            "peak_kind": f"bf16 dense sustained ({peaks['source']}): kernels timed inside the step"}
     roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["frac_of_burst"] = roof["achieved"] / peaks["bf16_tflops"]
     kernels = {
         "scas_calibration_attention": {"ms_per_step": ph["calib"] * 1e3 / K, "tflops": calib_tflops,
                                        "frac_of_bf16_peak": calib_tflops / peaks["bf16_tflops_sustained"]},
@@ -1023,6 +1221,7 @@ def main():
 
     # ------------------------------------------------ int8 retained cache
     quant = int8_cache(pipe, max_over_ranks, ph["attn"] * 1e3 / K, peaks["hbm_gbs"]) if args.quant else None
+    quant4 = int4_cache(pipe, max_over_ranks, ph["attn"] * 1e3 / K, peaks["hbm_gbs"]) if args.quant else None
 
     # ------------------------------------------------ generation order (scale by scale)
     gen = None
@@ -1051,7 +1250,13 @@ def main():
         dt = time.perf_counter() - t0
         cores = max([x.get("num_threads", 1) for x in threadpool_info()] or [1])
         cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-               "sample": sample.describe() + f"; {n} repetitions, {dt:.1f} s"}
+               "sample": sample.describe() + f"; {n} repetitions, {dt:.1f} s", "per_step": sample.per_step()}
+
+    # A compact copy of the per-kernel figures inside `roofline`, so that they
+    # travel with the headline fields.  Convention: kernels timed inside the
+    # step are set against the sustained bf16 peak, single launches timed
+    # alone against the burst peak; both fractions are given for each.
+    roof["per_kernel"] = summarize_kernels(kernels, quant, quant4, others, scas_o, peaks)
 
     if rank == 0:
         line = {
@@ -1061,7 +1266,7 @@ def main():
             "config": arm_config(w, world),
             "pruned_attention_tflops": pruned_tflops, "query_tokens_per_s": qtok_s, "compaction_gbs": comp_gbs,
             "roofline": roof, "kernels": kernels, "generation_order": gen, "ranking_stability": stab,
-            "int8_cache": quant, "other_configs": others, "scas_without_output": scas_o,
+            "int8_cache": quant, "int4_cache": quant4, "other_configs": others, "scas_without_output": scas_o,
             "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches,
             "clocks": clk, "peaks": peaks,

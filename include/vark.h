@@ -107,6 +107,9 @@ int vark_version(void);
  *              the mass is the same up to fp32 summation order).
  *   dev_status dev  int32, required; the caller sets it to 0 before the call;
  *              a kernel that gives up a bounded wait stores VARK_E_TIMEOUT.
+ * Limits: the per-row mass partials of S scales live in shared memory, so
+ *   with D = 128 at most 30 scales fit the 227 KB a CTA may use (D = 64: all
+ *   VARK_MAX_SCALES); more return VARK_E_SHAPE before any device call.
  * Errors: VARK_E_ARG, VARK_E_SHAPE, VARK_E_ALIGN, VARK_E_CUDA, VARK_E_DEVICE.
  */
 int vark_scas_accumulate(const uint16_t* q, const uint16_t* k, const uint16_t* v,
@@ -143,6 +146,8 @@ int vark_scas_finalize(const float* mass, int L, int H, int S, int n_calls, doub
  *   budget_bp  budget in basis points of F, 0..10000 (10000 keeps everything).
  *   n_sinks    number of leading sink scales never dropped, 0..S.
  *   keep       host uint8 [L][H][S] output, 1 = retained.
+ * Limits: L * H <= 2^24 and F * 10000 < 2^63 (the budget test is exact int64
+ *   arithmetic); larger shapes return VARK_E_SHAPE before scas is read.
  * Errors: VARK_E_ARG (null, non-finite scas, budget > 10000), VARK_E_SHAPE,
  *         VARK_E_BUDGET (the sinks alone exceed the budget; keep untouched).
  */
@@ -266,6 +271,7 @@ int vark_pruned_attention_step(const uint16_t* q, const uint16_t* kc, const uint
  *   bytes  host int64 [S][L]: bytes[k][l] = retained K + V bytes (bf16) held
  *          after layer l during scale k; bytes[S-1][L-1] = 2 * 2 * layer_base[L].
  *   keep   host uint8 [L][H][S].
+ * Limits: L * H * T * B * D * 4 < 2^63.
  * Errors: VARK_E_ARG, VARK_E_SHAPE.
  */
 int vark_cache_size_after_layer(const uint8_t* keep, int L, int H, int S, const int32_t* sides, int B, int D,
@@ -283,6 +289,7 @@ int vark_cache_size_after_layer(const uint8_t* keep, int L, int H, int S, const 
  *   drop_jaccard  |D_a & D_b| / |D_a | D_b| of the pairs each run's
  *                 vark_build_schedule drops at budget_bp (1 if neither drops).
  *   scas_a, scas_b  host fp64 [L][H][S], finite.
+ * Limits: as vark_build_schedule.
  * Errors: VARK_E_ARG, VARK_E_SHAPE (n_sinks >= S), VARK_E_BUDGET.
  */
 int vark_rank_stability(const double* scas_a, const double* scas_b, int L, int H, int S, const int32_t* sides,
@@ -308,7 +315,7 @@ int vark_rank_stability(const double* scas_a, const double* scas_b, int L, int H
  *   prefix_len  host int32 [S] out: N_k (0 while no non-sink scale exists).
  *   evict_step  host uint8 [L][H][S] out: first step k >= i at which (l, h, i)
  *               must be absent, 255 if it stays to the end (always 255 for
- *               sink scales).  S <= 254.
+ *               sink scales).  S <= 254, L * H <= INT32_MAX, F * 10000 < 2^63.
  * Errors: VARK_E_ARG, VARK_E_SHAPE, VARK_E_BUDGET (sinks alone over budget).
  */
 int vark_build_early_pruning_schedule(const double* scas, int L, int H, int S, const int32_t* sides,
@@ -374,6 +381,51 @@ int vark_quantize_kv_int8(const uint16_t* k, const uint16_t* v, int64_t layer_st
 int vark_dequantize_layer_int8(const int8_t* kq, const int8_t* vq, const float* k_absmax, const float* v_absmax,
                                int64_t kc_rows, int B, int H, int S, int D, const int32_t* sides,
                                const int32_t* head_off, const int32_t* seg_off,
+                               uint16_t* kc, uint16_t* vc, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Quantised retained cache (4-bit).  [VAR-Q] summary page: INT4 codes on the
+ * same (block, channel) groups keep BF16 quality, and bit packing turns the
+ * nominal bit width into real memory savings.  Same groups as the 8-bit cache;
+ * per channel:
+ *   a    = max |x| over the block        s = bf16(a / 7)   (IEEE fp32 division, RNE to bf16)
+ *   code = rint(x / s) in [-7, 7]        (IEEE fp32 division, half to even; s = 0 gives 0)
+ *   x'   = bf16(code * s)                (the product is exact in fp32; one rounding)
+ * Packing: nibble = code + 8 (1..15); the 8 channels c0..c7 of a row that
+ * start at a multiple of 8 form one little-endian 32-bit word, c0, c2, c4, c6
+ * in nibbles 0-3 and c1, c3, c5, c7 in nibbles 4-7.  Element e of the
+ * compacted layout (see the layout block) is nibble e % 8 of word e / 8, so a
+ * layer's codes start at byte layer_base[l] / 2 and a row is D / 2 bytes.
+ * Scale tables are [L][B][H][S][D] bf16 bits (0 for dropped scales).
+ * ------------------------------------------------------------------------- */
+
+/*
+ * vark_quantize_kv_int4 -- device.  Compaction with 4-bit quantisation: like
+ * vark_quantize_kv_int8, but kq / vq receive packed nibbles (layer_base[L] / 2
+ * bytes each) and k_scale / v_scale the bf16 scales s.  Each kept block is read
+ * from HBM once (as vark_quantize_kv_int8).  k, v, kq, vq, k_scale, v_scale
+ * 16-byte aligned; layer_stride a multiple of 8.
+ * Errors: VARK_E_ARG, VARK_E_SHAPE (D % 8 != 0, D > 512, H > 2048), VARK_E_ALIGN,
+ * VARK_E_CUDA.
+ */
+int vark_quantize_kv_int4(const uint16_t* k, const uint16_t* v, int64_t layer_stride,
+                          int L, int B, int H, int S, int D, const int32_t* sides,
+                          const uint8_t* keep, const int32_t* head_off, const int32_t* seg_off,
+                          const int64_t* layer_base, uint8_t* kq, uint8_t* vq,
+                          uint16_t* k_scale, uint16_t* v_scale, void* stream);
+
+/*
+ * vark_dequantize_layer_int4 -- device.  Expands one layer's 4-bit codes to
+ * its bf16 compacted block (as vark_dequantize_layer_int8).
+ *   kq, vq        dev uint8, the layer's packed codes (kq + layer_base[l] / 2),
+ *                 kc_rows rows of D / 2 bytes; 4-byte aligned.
+ *   k_scale, v_scale  dev bf16 bits [B][H][S][D], the layer's scale tables.
+ *   other arguments as vark_dequantize_layer_int8.
+ * Errors: as vark_dequantize_layer_int8.
+ */
+int vark_dequantize_layer_int4(const uint8_t* kq, const uint8_t* vq, const uint16_t* k_scale,
+                               const uint16_t* v_scale, int64_t kc_rows, int B, int H, int S, int D,
+                               const int32_t* sides, const int32_t* head_off, const int32_t* seg_off,
                                uint16_t* kc, uint16_t* vc, void* stream);
 
 #ifdef __cplusplus

@@ -56,6 +56,8 @@ _SIGNATURES = {
     "vark_recompact_kv": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P, _P, _P]),
     "vark_quantize_kv_int8": (_I, [_P, _P, _I64, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "vark_dequantize_layer_int8": (_I, [_P, _P, _P, _P, _I64, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
+    "vark_quantize_kv_int4": (_I, [_P, _P, _I64, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "vark_dequantize_layer_int4": (_I, [_P, _P, _P, _P, _I64, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
 }
 
 
@@ -110,6 +112,31 @@ def _dptr(t, dtype=None, name="tensor"):
     return t.data_ptr()
 
 
+def _need(t, name, shape=None, numel=None, at_least=None):
+    """Size check of a tensor argument against the shape the C call is given,
+    made before any pointer is taken: a mismatch would otherwise send the
+    kernels' tensor maps, atomics or stores outside the allocation."""
+    if t is None:
+        return
+    got = tuple(t.shape)
+    if shape is not None and got != tuple(int(x) for x in shape):
+        raise ValueError(f"{name}: shape {got}, expected {tuple(int(x) for x in shape)}")
+    if numel is not None and t.numel() != int(numel):
+        raise ValueError(f"{name}: {t.numel()} elements, expected {int(numel)}")
+    if at_least is not None and t.numel() < int(at_least):
+        raise ValueError(f"{name}: {t.numel()} elements, at least {int(at_least)} needed")
+
+
+def _tokens(sides):
+    return int(sum(int(x) * int(x) for x in sides))
+
+
+def _dims(t, n, name):
+    if t is None or len(t.shape) != n:
+        raise ValueError(f"{name} must have {n} dimensions")
+    return tuple(int(x) for x in t.shape)
+
+
 def _stream(stream):
     import torch
     if stream is None:
@@ -131,7 +158,16 @@ def vark_scas_accumulate(q, k, v, sides, tau, bias, mass, out=None, dev_status=N
     [B][H][T][D]; tau fp32 [H]; bias fp32 [H][S] or None; mass fp32 [H][S][S]
     accumulated; out bf16 like q or None; dev_status int32 [1]."""
     import torch
-    B, H, T, D = q.shape
+    B, H, T, D = _dims(q, 4, "q")
+    S = len(sides)
+    if T != _tokens(sides):
+        raise ValueError(f"q: {T} rows per (batch, head), the scale list has {_tokens(sides)} tokens")
+    for t, nm in ((k, "k"), (v, "v"), (out, "out")):
+        _need(t, nm, shape=(B, H, T, D))
+    _need(tau, "tau", numel=H)
+    _need(bias, "bias", numel=H * S)
+    _need(mass, "mass", numel=H * S * S)
+    _need(dev_status, "dev_status", at_least=1)
     s_arr, s_ptr = _sides_arg(sides)
     rc = _load().vark_scas_accumulate(
         _dptr(q, torch.bfloat16, "q"), _dptr(k, torch.bfloat16, "k"), _dptr(v, torch.bfloat16, "v"),
@@ -166,7 +202,13 @@ def vark_build_schedule(scas: np.ndarray, sides, budget_bp: int, n_sinks: int) -
 def vark_build_offsets(keep, sides, B: int, D: int, head_off, seg_off, past_len, layer_base, stream=None):
     """Device: offset tables into caller-provided int32/int64 tensors."""
     import torch
-    L, H, S = keep.shape
+    L, H, S = _dims(keep, 3, "keep")
+    if S != len(sides):
+        raise ValueError(f"keep has {S} scales, the scale list {len(sides)}")
+    _need(head_off, "head_off", numel=L * H)
+    _need(seg_off, "seg_off", numel=L * H * S)
+    _need(past_len, "past_len", numel=L * H * S)
+    _need(layer_base, "layer_base", numel=L + 1)
     s_arr, s_ptr = _sides_arg(sides)
     rc = _load().vark_build_offsets(
         _dptr(keep, torch.uint8, "keep"), L, H, S, s_ptr, int(B), int(D),
@@ -175,10 +217,29 @@ def vark_build_offsets(keep, sides, B: int, D: int, head_off, seg_off, past_len,
     _check(rc, "vark_build_offsets")
 
 
+def _layer_tables(keep, head_off, seg_off, layer_base, L, H, sides):
+    S = len(sides)
+    _need(keep, "keep", numel=L * H * S)
+    _need(head_off, "head_off", numel=L * H)
+    _need(seg_off, "seg_off", numel=L * H * S)
+    _need(layer_base, "layer_base", numel=L + 1)
+
+
+def _dense_source(k, v, layer_stride, L, per_layer):
+    if int(layer_stride) < per_layer:
+        raise ValueError(f"layer_stride {layer_stride} < {per_layer} elements of one layer")
+    need = (int(L) - 1) * int(layer_stride) + per_layer
+    _need(k, "k", at_least=need)
+    _need(v, "v", at_least=need)
+
+
 def vark_compact_kv(k, v, layer_stride: int, L: int, B: int, H: int, sides, D: int, keep, head_off, seg_off,
                     layer_base, kc, vc, stream=None):
-    """Device: gather retained scale blocks of all layers into kc / vc."""
+    """Device: gather retained scale blocks of all layers into kc / vc (each
+    must hold layer_base[L] elements)."""
     import torch
+    _layer_tables(keep, head_off, seg_off, layer_base, L, H, sides)
+    _dense_source(k, v, layer_stride, L, B * H * _tokens(sides) * D)
     s_arr, s_ptr = _sides_arg(sides)
     rc = _load().vark_compact_kv(
         _dptr(k, torch.bfloat16, "k"), _dptr(v, torch.bfloat16, "v"), int(layer_stride), int(L), int(B), int(H),
@@ -188,12 +249,38 @@ def vark_compact_kv(k, v, layer_stride: int, L: int, B: int, H: int, sides, D: i
     _check(rc, "vark_compact_kv")
 
 
+def _pruned_common_sizes(q, out, kc, vc, kc_rows, head_off, seg_off, past_len, tau, bias, dev_status, qshape,
+                         H, S):
+    _need(q, "q", shape=qshape)
+    _need(out, "out", shape=qshape)
+    if int(kc_rows) < 0 or int(kc_rows) % qshape[0] != 0:
+        raise ValueError(f"kc_rows {kc_rows} must be a non-negative multiple of the batch")
+    if int(kc_rows) > 0:
+        if kc is None or vc is None:
+            raise ValueError("kc and vc are required when kc_rows > 0")
+        _need(kc, "kc", at_least=int(kc_rows) * qshape[3])
+        _need(vc, "vc", at_least=int(kc_rows) * qshape[3])
+    _need(head_off, "head_off", numel=H)
+    _need(seg_off, "seg_off", numel=H * S)
+    _need(past_len, "past_len", numel=H * S)
+    _need(tau, "tau", numel=H)
+    _need(bias, "bias", numel=H * S)
+    _need(dev_status, "dev_status", at_least=1)
+
+
 def vark_pruned_attention(q, kc, vc, kc_rows: int, k_dense, v_dense, sides, query_scale: int, head_off, seg_off,
                           past_len, tau, bias, out, dev_status, stream=None):
     """Device: pruned-cache attention of one layer (see vark.h)."""
     import torch
-    B, H = k_dense.shape[0], k_dense.shape[1]
-    D = k_dense.shape[3]
+    B, H, T, D = _dims(k_dense, 4, "k_dense")
+    if T != _tokens(sides):
+        raise ValueError(f"k_dense: {T} rows per (batch, head), the scale list has {_tokens(sides)} tokens")
+    if not -1 <= int(query_scale) < len(sides):
+        raise ValueError(f"query_scale {query_scale} out of range")
+    Tq = T if int(query_scale) < 0 else int(sides[query_scale]) ** 2
+    _need(v_dense, "v_dense", shape=(B, H, T, D))
+    _pruned_common_sizes(q, out, kc, vc, kc_rows, head_off, seg_off, past_len, tau, bias, dev_status,
+                         (B, H, Tq, D), H, len(sides))
     s_arr, s_ptr = _sides_arg(sides)
     kcp = kc.data_ptr() if (kc is not None and kc_rows > 0) else None
     vcp = vc.data_ptr() if (vc is not None and kc_rows > 0) else None
@@ -215,6 +302,10 @@ def vark_append_scale(k_new, v_new, layer_stride: int, L: int, B: int, H: int, s
                       head_off, seg_off, layer_base, kc, vc, stream=None):
     """Device: append scale `scale` of every layer to the compacted cache."""
     import torch
+    if not 0 <= int(scale) < len(sides):
+        raise ValueError(f"scale {scale} out of range")
+    _layer_tables(keep, head_off, seg_off, layer_base, L, H, sides)
+    _dense_source(k_new, v_new, layer_stride, L, B * H * int(sides[scale]) ** 2 * D)
     s_arr, s_ptr = _sides_arg(sides)
     rc = _load().vark_append_scale(
         _dptr(k_new, torch.bfloat16, "k_new"), _dptr(v_new, torch.bfloat16, "v_new"), int(layer_stride), int(L),
@@ -229,7 +320,12 @@ def vark_pruned_attention_step(q, kc, vc, kc_rows: int, k_local, v_local, sides,
                                past_len, tau, bias, out, dev_status, stream=None):
     """Device: pruned attention for the queries of the scale being generated."""
     import torch
-    B, H, _, D = k_local.shape
+    B, H, nk, D = _dims(k_local, 4, "k_local")
+    if not 0 <= int(scale) < len(sides) or nk != int(sides[scale]) ** 2:
+        raise ValueError(f"k_local holds {nk} rows per (batch, head), scale {scale} has a different size")
+    _need(v_local, "v_local", shape=(B, H, nk, D))
+    _pruned_common_sizes(q, out, kc, vc, kc_rows, head_off, seg_off, past_len, tau, bias, dev_status,
+                         (B, H, nk, D), H, len(sides))
     s_arr, s_ptr = _sides_arg(sides)
     kcp = kc.data_ptr() if (kc is not None and kc_rows > 0) else None
     vcp = vc.data_ptr() if (vc is not None and kc_rows > 0) else None
@@ -287,8 +383,14 @@ def vark_build_early_pruning_schedule(scas: np.ndarray, sides, budget_bp: int, n
 def vark_recompact_kv(kc_old, vc_old, head_off_old, seg_off_old, layer_base_old, L: int, B: int, H: int, sides,
                       D: int, max_scale: int, keep_new, head_off_new, seg_off_new, layer_base_new, kc_new, vc_new,
                       stream=None):
-    """Device: move a compacted cache into the layout of a new retained set."""
+    """Device: move a compacted cache into the layout of a new retained set
+    (kc_new / vc_new must hold layer_base_new[L] elements)."""
     import torch
+    S = len(sides)
+    _need(head_off_old, "head_off_old", numel=L * H)
+    _need(seg_off_old, "seg_off_old", numel=L * H * S)
+    _need(layer_base_old, "layer_base_old", numel=L + 1)
+    _layer_tables(keep_new, head_off_new, seg_off_new, layer_base_new, L, H, sides)
     s_arr, s_ptr = _sides_arg(sides)
     rc = _load().vark_recompact_kv(
         _dptr(kc_old, torch.bfloat16, "kc_old"), _dptr(vc_old, torch.bfloat16, "vc_old"),
@@ -302,8 +404,13 @@ def vark_recompact_kv(kc_old, vc_old, head_off_old, seg_off_old, layer_base_old,
 
 def vark_quantize_kv_int8(k, v, layer_stride: int, L: int, B: int, H: int, sides, D: int, keep, head_off, seg_off,
                           layer_base, kq, vq, k_absmax, v_absmax, stream=None):
-    """Device: compaction into int8 codes + per-(block, channel) absmax."""
+    """Device: compaction into int8 codes + per-(block, channel) absmax (kq /
+    vq must hold layer_base[L] bytes)."""
     import torch
+    _layer_tables(keep, head_off, seg_off, layer_base, L, H, sides)
+    _dense_source(k, v, layer_stride, L, B * H * _tokens(sides) * D)
+    _need(k_absmax, "k_absmax", numel=L * B * H * len(sides) * D)
+    _need(v_absmax, "v_absmax", numel=L * B * H * len(sides) * D)
     s_arr, s_ptr = _sides_arg(sides)
     rc = _load().vark_quantize_kv_int8(
         _dptr(k, torch.bfloat16, "k"), _dptr(v, torch.bfloat16, "v"), int(layer_stride), int(L), int(B), int(H),
@@ -318,6 +425,13 @@ def vark_dequantize_layer_int8(kq, vq, k_absmax, v_absmax, kc_rows: int, B: int,
                                seg_off, kc, vc, stream=None):
     """Device: one layer's int8 codes back to its bf16 compacted block."""
     import torch
+    S = len(sides)
+    for t, nm in ((kq, "kq"), (vq, "vq"), (kc, "kc"), (vc, "vc")):
+        _need(t, nm, at_least=int(kc_rows) * D)
+    _need(k_absmax, "k_absmax", numel=B * H * S * D)
+    _need(v_absmax, "v_absmax", numel=B * H * S * D)
+    _need(head_off, "head_off", numel=H)
+    _need(seg_off, "seg_off", numel=H * S)
     s_arr, s_ptr = _sides_arg(sides)
     rc = _load().vark_dequantize_layer_int8(
         _dptr(kq, torch.int8, "kq"), _dptr(vq, torch.int8, "vq"), _dptr(k_absmax, torch.float32, "k_absmax"),
@@ -325,3 +439,45 @@ def vark_dequantize_layer_int8(kq, vq, k_absmax, v_absmax, kc_rows: int, B: int,
         _dptr(head_off, torch.int32, "head_off"), _dptr(seg_off, torch.int32, "seg_off"),
         _dptr(kc, torch.bfloat16, "kc"), _dptr(vc, torch.bfloat16, "vc"), _stream(stream))
     _check(rc, "vark_dequantize_layer_int8")
+
+
+def vark_quantize_kv_int4(k, v, layer_stride: int, L: int, B: int, H: int, sides, D: int, keep, head_off, seg_off,
+                          layer_base, kq, vq, k_scale, v_scale, stream=None):
+    """Device: compaction into packed 4-bit codes + per-(block, channel) bf16
+    scales (kq / vq must hold layer_base[L] / 2 bytes)."""
+    import torch
+    _layer_tables(keep, head_off, seg_off, layer_base, L, H, sides)
+    _dense_source(k, v, layer_stride, L, B * H * _tokens(sides) * D)
+    _need(k_scale, "k_scale", numel=L * B * H * len(sides) * D)
+    _need(v_scale, "v_scale", numel=L * B * H * len(sides) * D)
+    s_arr, s_ptr = _sides_arg(sides)
+    rc = _load().vark_quantize_kv_int4(
+        _dptr(k, torch.bfloat16, "k"), _dptr(v, torch.bfloat16, "v"), int(layer_stride), int(L), int(B), int(H),
+        len(s_arr), int(D), s_ptr, _dptr(keep, torch.uint8, "keep"), _dptr(head_off, torch.int32, "head_off"),
+        _dptr(seg_off, torch.int32, "seg_off"), _dptr(layer_base, torch.int64, "layer_base"),
+        _dptr(kq, torch.uint8, "kq"), _dptr(vq, torch.uint8, "vq"), _dptr(k_scale, torch.int16, "k_scale"),
+        _dptr(v_scale, torch.int16, "v_scale"), _stream(stream))
+    _check(rc, "vark_quantize_kv_int4")
+
+
+def vark_dequantize_layer_int4(kq, vq, k_scale, v_scale, kc_rows: int, B: int, H: int, sides, D: int, head_off,
+                               seg_off, kc, vc, stream=None):
+    """Device: one layer's packed 4-bit codes back to its bf16 compacted block."""
+    import torch
+    S = len(sides)
+    _need(kq, "kq", at_least=int(kc_rows) * D // 2)
+    _need(vq, "vq", at_least=int(kc_rows) * D // 2)
+    for t, nm in ((kc, "kc"), (vc, "vc")):
+        _need(t, nm, at_least=int(kc_rows) * D)
+    _need(k_scale, "k_scale", numel=B * H * S * D)
+    _need(v_scale, "v_scale", numel=B * H * S * D)
+    _need(head_off, "head_off", numel=H)
+    _need(seg_off, "seg_off", numel=H * S)
+    s_arr, s_ptr = _sides_arg(sides)
+    rc = _load().vark_dequantize_layer_int4(
+        _dptr(kq, torch.uint8, "kq"), _dptr(vq, torch.uint8, "vq"), _dptr(k_scale, torch.int16, "k_scale"),
+        _dptr(v_scale, torch.int16, "v_scale"), int(kc_rows), int(B), int(H), len(s_arr), int(D), s_ptr,
+        _dptr(head_off, torch.int32, "head_off"), _dptr(seg_off, torch.int32, "seg_off"),
+        _dptr(kc, torch.bfloat16, "kc"), _dptr(vc, torch.bfloat16, "vc"), _stream(stream))
+    _check(rc, "vark_dequantize_layer_int4")
+

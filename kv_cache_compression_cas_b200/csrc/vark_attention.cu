@@ -93,6 +93,13 @@ struct Params {
   int withhold_tile;
 };
 
+// P_X is written and consumed in kPChunks column chunks of kBlockN / kPChunks
+// keys: the softmax stores a chunk as soon as its exponentials are done and
+// the MMA thread issues that chunk's share of PV_X at once, so PV_X overlaps
+// the rest of the softmax instead of following it.
+constexpr int kPChunks = 4;
+constexpr int kChunkKeys = kBlockN / kPChunks;   // 32 keys = 16 TMEM columns of bf16 pairs
+
 enum Bar {
   kBarQ = 0,
   kBarKFull = 1,      // [2]
@@ -100,10 +107,10 @@ enum Bar {
   kBarKEmpty = 5,     // [2]
   kBarVEmpty = 7,     // [2]
   kBarSFull = 9,      // [tile]
-  kBarPFull = 11,     // [tile]
-  kBarODone = 13,     // [tile]
-  kBarDrain = 15,
-  kNumBars = 16
+  kBarPFull = 11,     // [tile][kPChunks]; without O, chunk 0 = "S_X read"
+  kBarODone = 19,     // [tile]
+  kBarDrain = 21,
+  kNumBars = 22
 };
 
 template <int D>
@@ -303,7 +310,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(bar(kBarSFull + x), 1);
-      mbar_init(bar(kBarPFull + x), kBlockM);
+      for (int c = 0; c < kPChunks; ++c) mbar_init(bar(kBarPFull + x * kPChunks + c), kBlockM / 32);  // one arrival per warp
       mbar_init(bar(kBarODone + x), 1);
     }
     mbar_init(bar(kBarDrain), 1);
@@ -356,9 +363,16 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       // ---------------------------------------------------------- producer
       // (Q and the first kStages key tiles were issued right after the
       // barrier initialisation, by this same thread.)
-      int issued_k = min(min(n, kStages), p.withhold_tile < 0 ? n : p.withhold_tile);
-      int issued_v = WITH_O ? issued_k : 0;
-      for (int j = issued_k; j < n; ++j) {
+      // last tile this thread loaded into each stage (-1: none); only those
+      // loads can still be in flight when the loop ends
+      const int first = min(min(n, kStages), p.withhold_tile < 0 ? n : p.withhold_tile);
+      int last_k[kStages], last_v[kStages];
+      for (int st = 0; st < kStages; ++st) {
+        const bool mine = st < first;
+        last_k[st] = mine ? st : -1;
+        last_v[st] = (mine && WITH_O) ? st : -1;
+      }
+      for (int j = first; j < n; ++j) {
         const int st = j % kStages;
         const KTile t = it.tile(p, j);
         if (j == p.withhold_tile) break;   // test hook: this tile never arrives
@@ -369,7 +383,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           if (t.src == 0) tma_load_3d(dst, &tm_k, bar(kBarKFull + st), c * 64, t.row, it.bh);
           else tma_load_2d(dst, &tm_kc, bar(kBarKFull + st), c * 64, t.row);
         }
-        issued_k = j + 1;
+        last_k[st] = j;
         if (!WITH_O) continue;
         if (j >= kStages && !mbar_wait(bar(kBarVEmpty + st), ((j / kStages) - 1) & 1, abort_flag, p.status, p.wait_limit_ns)) break;
         mbar_arrive_expect_tx(bar(kBarVFull + st), kTileBytes);
@@ -378,16 +392,16 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           if (t.src == 0) tma_load_3d(dst, &tm_v, bar(kBarVFull + st), c * 64, t.row, it.bh);
           else tma_load_2d(dst, &tm_vc, bar(kBarVFull + st), c * 64, t.row);
         }
-        issued_v = j + 1;
+        last_v[st] = j;
       }
       // Drain: every load issued here has landed before the CTA exits
       // (immediate on the normal path; bounded on the abort path).
       volatile int no_abort = 0;
       mbar_wait(bar(kBarQ), 0, &no_abort, nullptr);
-      for (int j = max(0, issued_k - kStages); j < issued_k; ++j)
-        mbar_wait(bar(kBarKFull + j % kStages), (j / kStages) & 1, &no_abort, nullptr);
-      for (int j = max(0, issued_v - kStages); j < issued_v; ++j)
-        mbar_wait(bar(kBarVFull + j % kStages), (j / kStages) & 1, &no_abort, nullptr);
+      for (int st = 0; st < kStages; ++st) {
+        if (last_k[st] >= 0) mbar_wait(bar(kBarKFull + st), (last_k[st] / kStages) & 1, &no_abort, nullptr);
+        if (last_v[st] >= 0) mbar_wait(bar(kBarVFull + st), (last_v[st] / kStages) & 1, &no_abort, nullptr);
+      }
     } else if (warp == 1 && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
       constexpr uint32_t idesc_s = idesc_bf16_f32(kBlockM, kBlockN, false, false);
@@ -401,12 +415,23 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           mma_bf16_ss(tmem + x * kBlockN, a, b, idesc_s, kk > 0 ? 1u : 0u);
         }
       };
-      auto issue_pv = [&](int x, int st, bool first) {
+      // PV_X of key tile jp from the V stage pst, one P chunk at a time: each
+      // chunk's two K = 16 steps are issued as soon as the softmax has stored
+      // that chunk.  Returns false on abort.
+      auto issue_pv = [&](int x, int pst, int jp) -> bool {
 #pragma unroll
-        for (int kk = 0; kk < kBlockN / 16; ++kk) {
-          const uint64_t b = smem_desc_sw128(sV + st * kTileBytes + kk * 2048, kPanelBytes, 1024);
-          mma_bf16_ts(tmem + 256 + x * D, tmem + x * kBlockN + kk * 8, b, idesc_o, (!first || kk > 0) ? 1u : 0u);
+        for (int c = 0; c < kPChunks; ++c) {
+          if (!mbar_wait(bar(kBarPFull + x * kPChunks + c), jp & 1, abort_flag, p.status, p.wait_limit_ns))
+            return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kq = 0; kq < kChunkKeys / 16; ++kq) {
+            const int kk = c * (kChunkKeys / 16) + kq;
+            const uint64_t b = smem_desc_sw128(sV + pst * kTileBytes + kk * 2048, kPanelBytes, 1024);
+            mma_bf16_ts(tmem + 256 + x * D, tmem + x * kBlockN + kk * 8, b, idesc_o, (jp > 0 || kk > 0) ? 1u : 0u);
+          }
         }
+        return true;
       };
       bool ok = mbar_wait(bar(kBarQ), 0, abort_flag, p.status, p.wait_limit_ns);
       if (!WITH_O) {
@@ -415,7 +440,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           const int st = j % kStages;
           if (!(ok = mbar_wait(bar(kBarKFull + st), (j / kStages) & 1, abort_flag, p.status, p.wait_limit_ns))) break;
           for (int x = 0; x < n_act; ++x) {
-            if (j > 0 && !(ok = mbar_wait(bar(kBarPFull + x), (j - 1) & 1, abort_flag, p.status, p.wait_limit_ns))) break;
+            if (j > 0 && !(ok = mbar_wait(bar(kBarPFull + x * kPChunks), (j - 1) & 1, abort_flag, p.status, p.wait_limit_ns))) break;
             tc_fence_after();
             issue_s(x, st);
             mma_commit(bar(kBarSFull + x));
@@ -430,9 +455,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         if (j > 0 && !(ok = mbar_wait(bar(kBarVFull + pst), ((j - 1) / kStages) & 1, abort_flag, p.status, p.wait_limit_ns))) break;
         for (int x = 0; x < n_act; ++x) {
           if (j > 0) {
-            if (!(ok = mbar_wait(bar(kBarPFull + x), (j - 1) & 1, abort_flag, p.status, p.wait_limit_ns))) break;
-            tc_fence_after();
-            issue_pv(x, pst, j == 1);
+            if (!(ok = issue_pv(x, pst, j - 1))) break;
           } else {
             tc_fence_after();
           }
@@ -447,9 +470,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         const int pst = (n - 1) % kStages;
         ok = mbar_wait(bar(kBarVFull + pst), ((n - 1) / kStages) & 1, abort_flag, p.status, p.wait_limit_ns);
         for (int x = 0; ok && x < n_act; ++x) {
-          if (!(ok = mbar_wait(bar(kBarPFull + x), (n - 1) & 1, abort_flag, p.status, p.wait_limit_ns))) break;
-          tc_fence_after();
-          issue_pv(x, pst, n == 1);
+          if (!(ok = issue_pv(x, pst, n - 1))) break;
           mma_commit(bar(kBarODone + x));
         }
       }
@@ -514,7 +535,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       }
       if (!WITH_O) {   // S_X is in registers: the next S MMA of this tile may overwrite it
         tc_fence_before();
-        mbar_arrive(bar(kBarPFull + x));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kBarPFull + x * kPChunks));
       }
       float m_tile, sh;
       if (fast) {
@@ -581,25 +603,49 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           tmem_st32(tO + c * 32, v);
         }
       }
-      // p = 2^(exponent - m_used)
-      if (fast) {
-        const float shm = sh - m_used;
+      // p = 2^(exponent - m_used), one chunk of kChunkKeys columns at a time.
+      // With O, chunk q's bf16 pairs go to TMEM (over S_X's first columns)
+      // while chunk q+1's exponentials run, and the warp signals the chunk
+      // to the MMA thread once its store has completed.
+      const float shm = fast ? sh - m_used : -m_used;
 #pragma unroll
-        for (int c = 0; c < kBlockN; c += 2) ffma2(sv[c], sv[c + 1], sv[c], sv[c + 1], qk2, qk2, shm, shm);
+      for (int q = 0; q < kPChunks; ++q) {
+        float* cv = sv + q * kChunkKeys;
+        if (fast) {
 #pragma unroll
-        for (int c = 0; c < kBlockN; c += 8) {
-          constexpr int kPoly = WITH_O ? kPolyPer8 : kPolyPer8NoO;
+          for (int c = 0; c < kChunkKeys; c += 2) ffma2(cv[c], cv[c + 1], cv[c], cv[c + 1], qk2, qk2, shm, shm);
 #pragma unroll
-          for (int i = 0; i < kPoly; i += 2) exp2_poly2(sv[c + i], sv[c + i + 1]);
+          for (int c = 0; c < kChunkKeys; c += 8) {
+            constexpr int kPoly = WITH_O ? kPolyPer8 : kPolyPer8NoO;
 #pragma unroll
-          for (int i = kPoly; i < 8; ++i) sv[c + i] = ex2_approx(sv[c + i]);
+            for (int i = 0; i < kPoly; i += 2) exp2_poly2(cv[c + i], cv[c + i + 1]);
+#pragma unroll
+            for (int i = kPoly; i < 8; ++i) cv[c + i] = ex2_approx(cv[c + i]);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < kChunkKeys; c += 2) fadd2(cv[c], cv[c + 1], cv[c], cv[c + 1], shm, shm);
+#pragma unroll
+          for (int c = 0; c < kChunkKeys; ++c) cv[c] = ex2_approx(cv[c]);
         }
-      } else {
-        const float shm = -m_used;
+        if (WITH_O) {
+          if (q > 0) {   // chunk q-1's store has been in flight during these exponentials
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kBarPFull + x * kPChunks + q - 1));
+          }
+          uint32_t pk[kChunkKeys / 2];
 #pragma unroll
-        for (int c = 0; c < kBlockN; c += 2) fadd2(sv[c], sv[c + 1], sv[c], sv[c + 1], shm, shm);
-#pragma unroll
-        for (int c = 0; c < kBlockN; ++c) sv[c] = ex2_approx(sv[c]);
+          for (int c = 0; c < kChunkKeys / 2; ++c) pk[c] = pack_bf16x2(cv[2 * c], cv[2 * c + 1]);
+          tmem_st16(tS + q * (kChunkKeys / 2), pk);
+        }
+      }
+      if (WITH_O) {
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kBarPFull + x * kPChunks + kPChunks - 1));
       }
       float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f, a4 = 0.f, a5 = 0.f, a6 = 0.f, a7 = 0.f;
 #pragma unroll
@@ -633,20 +679,6 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             named_bar_sync(3 + x, kBlockM);
           });
         }
-      }
-      // P_X (bf16 pairs) over the first 64 columns of S_X
-      if (WITH_O) {
-        uint32_t pk[2][32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          pk[0][c] = pack_bf16x2(sv[2 * c], sv[2 * c + 1]);
-          pk[1][c] = pack_bf16x2(sv[64 + 2 * c], sv[64 + 2 * c + 1]);
-        }
-        tmem_st32(tS, pk[0]);
-        tmem_st32(tS + 32, pk[1]);
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bar(kBarPFull + x));
       }
     }
 
@@ -778,6 +810,9 @@ static int launch(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap&
   return cudaGetLastError() == cudaSuccess ? VARK_OK : VARK_E_CUDA;
 }
 
+// Dynamic shared memory a CTA may opt into on sm_100 (227 KB).
+constexpr int kMaxSmemOptin = 232448;
+
 static bool finite_shape(int B, int H, int T, int D) {
   return B >= 1 && H >= 1 && int64_t(B) * H <= INT32_MAX / 2 && int64_t(B) * H * T * D < (int64_t(1) << 40);
 }
@@ -797,6 +832,8 @@ extern "C" int vark_scas_accumulate(const uint16_t* q, const uint16_t* k, const 
   if (rc) return rc;
   if (D != 64 && D != 128) return VARK_E_SHAPE;
   if (!finite_shape(B, H, lp.sc.T, D)) return VARK_E_SHAPE;
+  // the per-row mass partials of every scale must fit next to the tiles
+  if ((D == 128 ? Smem<128>::alloc(true, S) : Smem<64>::alloc(true, S)) > kMaxSmemOptin) return VARK_E_SHAPE;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || (out && !aligned16(out))) return VARK_E_ALIGN;
   if ((rc = check_device_sm100())) return rc;
   lp.B = B; lp.H = H;

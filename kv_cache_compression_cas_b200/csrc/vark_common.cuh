@@ -230,6 +230,16 @@ VARK_DEV void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
       : "memory");
 }
 
+// 32 lanes x 16 consecutive 32-bit columns (one chunk of a P tile).
+VARK_DEV void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
 VARK_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // tcgen05.ld writes its registers asynchronously; after tmem_wait_ld, pass the
@@ -308,8 +318,9 @@ VARK_DEV void fadd2(float& d0, float& d1, float a0, float a1, float b0, float b1
 // 2^x for a pair on the FMA pipe.  Range reduction x = n + f with
 // n = round(x) (adding 1.5 * 2^23 leaves n in the low mantissa bits), so
 // f = x - n lies in [-1/2, 1/2]; 2^f comes from the degree-3 minimax
-// polynomial in relative error (max 7.5e-5) fitted by csrc/fit_exp2.py, and
-// 2^n is added into the exponent field.  x is clamped below at -125 (results stay normal fp32 numbers).
+// polynomial in relative error (max 7.5e-5; Remez exchange, coefficients
+// rounded to fp32 -- tests/test_exp2_poly.py re-derives them), and 2^n is
+// added into the exponent field.  x is clamped below at -125 (results stay normal fp32 numbers).
 VARK_DEV void exp2_poly2(float& a, float& b) {
   constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
   constexpr float c0 = 0.9999280571937561f, c1 = 0.6932609677314758f;

@@ -8,6 +8,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
+#include <climits>
 #include <cstring>
 #include <vector>
 
@@ -41,6 +42,12 @@ static bool sides_ok(int S, const int32_t* sides, int64_t* T_out) {
   return true;
 }
 
+// The budget test compares kept * 10000 with budget_bp * F in int64, with
+// F = (L * H) * T tokens: both sides stay below 2^63 when F <= INT64_MAX / 10000.
+static bool budget_fits_int64(int64_t LH, int64_t T) {
+  return LH >= 1 && T >= 1 && LH <= INT64_MAX / 10000 / T;
+}
+
 extern "C" int vark_scas_finalize(const float* mass, int L, int H, int S, int n_calls, double* scas) {
   if (mass == nullptr || scas == nullptr || n_calls < 1) return VARK_E_ARG;
   if (L < 1 || H < 1 || S < 1 || S > VARK_MAX_SCALES) return VARK_E_SHAPE;
@@ -70,6 +77,7 @@ extern "C" int vark_build_schedule(const double* scas, int L, int H, int S, cons
   int64_t T = 0;
   if (L < 1 || H < 1 || !sides_ok(S, sides, &T) || n_sinks > S) return VARK_E_SHAPE;
   if (int64_t(L) * H > (int64_t(1) << 24)) return VARK_E_SHAPE;
+  if (!budget_fits_int64(int64_t(L) * H, T)) return VARK_E_SHAPE;
   const int64_t LHS = int64_t(L) * H * S;
   for (int64_t i = 0; i < LHS; ++i)
     if (!std::isfinite(scas[i])) return VARK_E_ARG;
@@ -116,6 +124,8 @@ extern "C" int vark_cache_size_after_layer(const uint8_t* keep, int L, int H, in
   if (keep == nullptr || bytes == nullptr || sides == nullptr) return VARK_E_ARG;
   int64_t T = 0;
   if (L < 1 || H < 1 || B < 1 || D < 1 || !sides_ok(S, sides, &T)) return VARK_E_SHAPE;
+  // every byte count is at most L * H * T * B * D * 4, which must fit int64
+  if (int64_t(L) * H > INT64_MAX / T / (int64_t(B) * D * 4)) return VARK_E_SHAPE;
   int64_t total = 0;
   const int64_t per_token = int64_t(B) * D * 2 * 2;   // K and V, bf16
   for (int k = 0; k < S; ++k) {
@@ -153,6 +163,7 @@ extern "C" int vark_rank_stability(const double* scas_a, const double* scas_b, i
   if (!scas_a || !scas_b || !sides || !spearman || !drop_jaccard) return VARK_E_ARG;
   int64_t T = 0;
   if (L < 1 || H < 1 || !sides_ok(S, sides, &T) || n_sinks < 0 || n_sinks >= S) return VARK_E_SHAPE;
+  if (int64_t(L) * H > (int64_t(1) << 24) || !budget_fits_int64(int64_t(L) * H, T)) return VARK_E_SHAPE;
   std::vector<double> a, b;
   for (int l = 0; l < L; ++l)
     for (int h = 0; h < H; ++h)
@@ -198,6 +209,8 @@ extern "C" int vark_build_early_pruning_schedule(const double* scas, int L, int 
   if (budget_bp > 10000u || n_sinks < 0) return VARK_E_ARG;
   int64_t T = 0;
   if (L < 1 || H < 1 || !sides_ok(S, sides, &T) || n_sinks > S || S > 254) return VARK_E_SHAPE;
+  // prefix lengths are int32; the budget arithmetic stays in int64
+  if (int64_t(L) * H > INT32_MAX || !budget_fits_int64(int64_t(L) * H, T)) return VARK_E_SHAPE;
   const int64_t LH = int64_t(L) * H;
   const int64_t LHS = LH * S;
   for (int64_t i = 0; i < LHS; ++i)

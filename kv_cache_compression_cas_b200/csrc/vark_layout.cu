@@ -13,6 +13,7 @@
 // and a walk over at most S scales.  Copies are 16-byte vectors, coalesced,
 // with several loads in flight per thread before the stores.
 #include <algorithm>
+#include <type_traits>
 
 #include "vark_common.cuh"
 
@@ -105,6 +106,7 @@ __device__ __forceinline__ void block_exclusive_scan(int32_t* a, int n, int32_t*
 
 constexpr int kChunkRows = 64;
 constexpr int kCompactThreads = 256;
+constexpr int kCompactInflight = 4;
 constexpr int kMaxGroupLH = 4096;   // (layer, head) pairs per launch group
 
 struct CompactParams {
@@ -206,11 +208,11 @@ __global__ void __launch_bounds__(kCompactThreads, 4) compact_kernel(
     }
     const int nvec = nrows * vec_per_row;
 
-    // 4 K + 4 V vectors in flight per thread, then the stores.
-    for (int base = 0; base < nvec; base += 4 * kCompactThreads) {
-      uint4 a[4], bq[4];
+    // kCompactInflight K + kCompactInflight V vectors in flight per thread, then the stores.
+    for (int base = 0; base < nvec; base += kCompactInflight * kCompactThreads) {
+      uint4 a[kCompactInflight], bq[kCompactInflight];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < kCompactInflight; ++u) {
         const int e = base + u * kCompactThreads + threadIdx.x;
         if (e < nvec) {
           a[u] = __ldcs(k + src_v + e);
@@ -218,7 +220,7 @@ __global__ void __launch_bounds__(kCompactThreads, 4) compact_kernel(
         }
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < kCompactInflight; ++u) {
         const int e = base + u * kCompactThreads + threadIdx.x;
         if (e < nvec) {
           __stcs(kc + dst_v + e, a[u]);
@@ -369,6 +371,8 @@ constexpr int kQuantCluster = 8;
 constexpr int kQuantGroupLH = 2048;  // (layer, head) pairs per launch group
 constexpr int kSmallRows = 1024;
 constexpr int kQuantMaxD = 512;
+// 0: single-read cluster kernel; 1: two streaming passes (absmax, then codes).
+constexpr bool kQuantTwoPass = false;
 
 struct QuantParams {
   ScaleTable sc;
@@ -422,15 +426,20 @@ __device__ __forceinline__ void absmax8(uint32_t (&acc)[4], const uint4& x) {
   acc[3] = __vmaxu2(acc[3], x.w & 0x7FFF7FFFu);
 }
 
-// Channel scale: sc = a / 127 (IEEE), and rc = RN(1 / sc) when the product
-// path is usable (2^-100 <= sc <= 2^100), else 0 (always divide).
+// Channel scale: 8-bit codes sc = a / 127 (IEEE); 4-bit codes sc = bf16(a / 7)
+// (IEEE division rounded to bf16, the value the 4-bit scale table stores);
+// rc = RN(1 / sc) when the product path is usable (2^-100 <= sc <= 2^100),
+// else 0 (always divide).
 struct QScale {
   float sc, rc;
 };
 
+__device__ __forceinline__ float round_to_bf16(float x) { return __uint_as_float(pack_bf16x2(x, 0.f) << 16); }
+
+template <int BITS>
 __device__ __forceinline__ QScale make_qscale(float a) {
   QScale q;
-  q.sc = a / 127.f;
+  q.sc = BITS == 8 ? a / 127.f : round_to_bf16(a / 7.f);
   q.rc = (q.sc >= 0x1p-100f && q.sc <= 0x1p100f) ? __frcp_rn(q.sc) : 0.f;
   return q;
 }
@@ -456,10 +465,15 @@ __device__ __forceinline__ uint32_t pack4_low_bytes(float y0, float y1, float y2
                      __byte_perm(__float_as_uint(y2), __float_as_uint(y3), 0x0040), 0x5410);
 }
 
-__device__ __forceinline__ uint2 codes8(const uint4& x, const float (&sc)[8], const float (&rc)[8], bool force) {
+// y[j] = kRound + rint(x_j / sc_j) for the 8 channels of one 16-byte vector.
+// With 8-bit codes |x / sc| <= 127 (1 + 2^-24); with 4-bit codes sc = bf16(a / 7)
+// >= (a / 7)(1 - 2^-8), so |x / sc| < 7.03: rint never leaves [-127, 127] /
+// [-7, 7] and no clamp is needed.
+__device__ __forceinline__ void code_sums8(const uint4& x, const float (&sc)[8], const float (&rc)[8], bool force,
+                                           float (&y)[8]) {
   const float v[8] = {lo_bf16(x.x), hi_bf16(x.x), lo_bf16(x.y), hi_bf16(x.y),
                       lo_bf16(x.z), hi_bf16(x.z), lo_bf16(x.w), hi_bf16(x.w)};
-  float y[8], d[8];   // y: kRound + rint(t); d > 1/2: t lies within |t| * 2^-20 of a half-integer
+  float d[8];         // d > 1/2: t lies within |t| * 2^-20 of a half-integer
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const float t = __fmul_rn(v[j], rc[j]);
@@ -473,16 +487,42 @@ __device__ __forceinline__ uint2 codes8(const uint4& x, const float (&sc)[8], co
     for (int j = 0; j < 8; ++j)
       if (force || d[j] > 0.5f) y[j] = __fadd_rn(sc[j] == 0.f ? 0.f : __fdiv_rn(v[j], sc[j]), kRound);
   }
+}
+
+// 8-bit codes: one byte per channel, in channel order.
+__device__ __forceinline__ uint2 codes8(const uint4& x, const float (&sc)[8], const float (&rc)[8], bool force) {
+  float y[8];
+  code_sums8(x, sc, rc, force, y);
   uint2 o;
   o.x = pack4_low_bytes(y[0], y[1], y[2], y[3]);
   o.y = pack4_low_bytes(y[4], y[5], y[6], y[7]);
   return o;
 }
 
+// 4-bit codes: nibble = code + 8; channels 0, 2, 4, 6 in nibbles 0-3 and 1, 3,
+// 5, 7 in nibbles 4-7 of one word (the low bits of kRound + code + 8 are the
+// nibble).  That order lets a consumer form bf16 pairs of adjacent channels
+// with one mask per pair.
+__device__ __forceinline__ uint32_t codes4x8(const uint4& x, const float (&sc)[8], const float (&rc)[8], bool force) {
+  float y[8];
+  code_sums8(x, sc, rc, force, y);
+  uint32_t w = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    w |= ((__float_as_uint(y[2 * j]) + 8u) & 0xFu) << (4 * j);
+    w |= ((__float_as_uint(y[2 * j + 1]) + 8u) & 0xFu) << (16 + 4 * j);
+  }
+  return w;
+}
+
+// BITS = 8: kq / vq int8 codes (one byte per element), ka / va fp32 absmax.
+// BITS = 4: kq / vq packed nibbles (one 32-bit word per 8 elements), ka / va
+// bf16 bits (uint16) of the scale bf16(a / 7).
+template <int BITS>
 __global__ void __cluster_dims__(kQuantCluster, 1, 1) __launch_bounds__(kQuantThreads, 5) quant_kernel(
     const uint4* __restrict__ k, const uint4* __restrict__ v, QuantParams p, const uint8_t* __restrict__ keep,
     const int32_t* __restrict__ head_off, const int32_t* __restrict__ seg_off, const int64_t* __restrict__ layer_base,
-    int8_t* __restrict__ kq, int8_t* __restrict__ vq, float* __restrict__ ka, float* __restrict__ va) {
+    void* __restrict__ kq, void* __restrict__ vq, void* __restrict__ ka, void* __restrict__ va) {
   __shared__ int32_t big_prefix[kQuantGroupLH + 1];
   __shared__ int32_t small_prefix[kQuantGroupLH + 1];
   __shared__ uint32_t keep_mask[kQuantGroupLH];
@@ -581,7 +621,7 @@ __global__ void __cluster_dims__(kQuantCluster, 1, 1) __launch_bounds__(kQuantTh
     }
     for (int x = threadIdx.x; x < dw; x += kQuantThreads) {   // the pair's scales, once per unit
       const uint32_t w = fin[x];
-      const QScale q0 = make_qscale(lo_bf16(w)), q1 = make_qscale(hi_bf16(w));
+      const QScale q0 = make_qscale<BITS>(lo_bf16(w)), q1 = make_qscale<BITS>(hi_bf16(w));
       fin_sc[2 * x] = q0.sc;
       fin_sc[2 * x + 1] = q1.sc;
       fin_rc[2 * x] = q0.rc;
@@ -605,27 +645,244 @@ __global__ void __cluster_dims__(kQuantCluster, 1, 1) __launch_bounds__(kQuantTh
       const int64_t R_l = (layer_base[q.l + 1] - layer_base[q.l]) / (int64_t(B) * D);
       const int64_t row0 =
           int64_t(q.b) * R_l + head_off[q.l * H + q.h] + seg_off[(int64_t(q.l) * H + q.h) * S + q.s];
-      uint2* dst = reinterpret_cast<uint2*>((q.t ? vq : kq) + layer_base[q.l] + (row0 + r_lo) * D) + cv;
+      // element index of this CTA's first row; 8 elements per 8-byte (int8) or 4-byte (int4) store
+      const int64_t e_first = layer_base[q.l] + (row0 + r_lo) * D;
       int32_t r = rg;
-      for (; r + 3 * nrg < nr; r += 4 * nrg) {
-        uint4 x[4];
+      if (BITS == 8) {
+        uint2* dst = reinterpret_cast<uint2*>(static_cast<int8_t*>(q.t ? vq : kq) + e_first) + cv;
+        for (; r + 3 * nrg < nr; r += 4 * nrg) {
+          uint4 x[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) x[e] = __ldcs(src + (r + e * nrg) * cv_n);
+          for (int e = 0; e < 4; ++e) x[e] = __ldcs(src + (r + e * nrg) * cv_n);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) dst[(r + e * nrg) * cv_n] = codes8(x[e], sc, rc, force);
+          for (int e = 0; e < 4; ++e) dst[(r + e * nrg) * cv_n] = codes8(x[e], sc, rc, force);
+        }
+        for (; r < nr; r += nrg) dst[r * cv_n] = codes8(__ldcs(src + r * cv_n), sc, rc, force);
+      } else {
+        uint32_t* dst = static_cast<uint32_t*>(q.t ? vq : kq) + e_first / 8 + cv;
+        for (; r + 3 * nrg < nr; r += 4 * nrg) {
+          uint4 x[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) x[e] = __ldcs(src + (r + e * nrg) * cv_n);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dst[(r + e * nrg) * cv_n] = codes4x8(x[e], sc, rc, force);
+        }
+        for (; r < nr; r += nrg) dst[r * cv_n] = codes4x8(__ldcs(src + r * cv_n), sc, rc, force);
       }
-      for (; r < nr; r += nrg) dst[r * cv_n] = codes8(__ldcs(src + r * cv_n), sc, rc, force);
     }
     // the block's absmax entries: once per block
     if (!big || rank == 0) {
-      float* ab = (q.t ? va : ka) + ((((int64_t(q.l) * B + q.b) * H + q.h) * S) + q.s) * D;
+      const int64_t t0 = ((((int64_t(q.l) * B + q.b) * H + q.h) * S) + q.s) * D;
       for (int c = threadIdx.x; c < D; c += kQuantThreads) {
         const uint32_t w = fin[c >> 1];
-        ab[c] = (c & 1) ? hi_bf16(w) : lo_bf16(w);
+        const float a = (c & 1) ? hi_bf16(w) : lo_bf16(w);
+        if (BITS == 8) static_cast<float*>(q.t ? va : ka)[t0 + c] = a;
+        else static_cast<uint16_t*>(q.t ? va : ka)[t0 + c] = uint16_t(__float_as_uint(make_qscale<4>(a).sc) >> 16);
       }
     }
   }
   cluster_sync_all();   // no CTA leaves while a peer may still read its partial maxima
+}
+
+// Two-pass quantisation.  Pass 1 (absmax_kernel): one CTA per (block,
+// tensor), big blocks first, streams the block once and writes its table
+// entries in their final form (fp32 absmax, or the bf16 scale of 4-bit codes)
+// -- no cross-CTA reduction, no atomics.  Pass 2 (codes_kernel): a pure stream
+// over (block, 64-row chunk) units in memory order, like the compaction; each
+// unit reads its 8 channels' table entries (L2-resident) and writes codes.
+// The kept bf16 bytes are read twice from HBM, but neither pass ever waits on
+// another CTA.
+constexpr int kAbsThreads = 256;
+constexpr int kCodeRows = 64;
+constexpr int kCodeThreads = 256;
+
+template <int BITS>
+__global__ void __launch_bounds__(kAbsThreads, 4) absmax_kernel(
+    const uint4* __restrict__ k, const uint4* __restrict__ v, QuantParams p, const uint8_t* __restrict__ keep,
+    void* __restrict__ ka, void* __restrict__ va) {
+  __shared__ int32_t big_prefix[kQuantGroupLH + 1];
+  __shared__ int32_t small_prefix[kQuantGroupLH + 1];
+  __shared__ uint32_t keep_mask[kQuantGroupLH];
+  __shared__ int32_t warp_tot[kAbsThreads / 32];
+  __shared__ __align__(16) uint32_t red[kAbsThreads * 4];
+  const int S = p.sc.S, H = p.H, D = p.D, B = p.B;
+  const int nlh = p.nl * H;
+  const int lh0 = p.l0 * H;
+  for (int i = threadIdx.x; i < nlh; i += kAbsThreads) {
+    const uint8_t* kp = keep + int64_t(lh0 + i) * S;
+    uint32_t m = 0;
+    for (int s = 0; s < S; ++s)
+      if (kp[s]) m |= 1u << s;
+    keep_mask[i] = m;
+    big_prefix[i] = __popc(m & p.big_mask);
+    small_prefix[i] = __popc(m & ~p.big_mask);
+  }
+  __syncthreads();
+  block_exclusive_scan<kAbsThreads, kQuantGroupLH>(big_prefix, nlh, warp_tot);
+  block_exclusive_scan<kAbsThreads, kQuantGroupLH>(small_prefix, nlh, warp_tot);
+  const int64_t n_big = int64_t(big_prefix[nlh]) * 2 * B;
+  const int64_t n_units = n_big + int64_t(small_prefix[nlh]) * 2 * B;
+  const int cv_n = D / 8;
+  const int nrg = kAbsThreads / cv_n;
+  const bool active = threadIdx.x < nrg * cv_n;
+  const int cv = threadIdx.x % cv_n;
+  const int rg = threadIdx.x / cv_n;
+  for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x) {
+    const bool big = u < n_big;
+    const QBlock q = big ? decode_block(u, big_prefix, keep_mask, p.big_mask, p)
+                         : decode_block(u - n_big, small_prefix, keep_mask, ~p.big_mask, p);
+    const int32_t nr = p.sc.n[q.s];
+    const uint4* src = (q.t ? v : k) +
+                       (int64_t(q.l) * p.layer_stride + ((int64_t(q.b) * H + q.h) * p.sc.T + p.sc.off[q.s]) * D) / 8 +
+                       cv;
+    uint32_t acc[4] = {0u, 0u, 0u, 0u};
+    if (active) {
+      int32_t r = rg;
+      for (; r + 7 * nrg < nr; r += 8 * nrg) {
+        uint4 x[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = __ldcs(src + int64_t(r + e * nrg) * cv_n);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) absmax8(acc, x[e]);
+      }
+      for (; r < nr; r += nrg) absmax8(acc, __ldcs(src + int64_t(r) * cv_n));
+      *reinterpret_cast<uint4*>(&red[threadIdx.x * 4]) = make_uint4(acc[0], acc[1], acc[2], acc[3]);
+    }
+    __syncthreads();
+    const int dw = D / 2;
+    const int64_t t0 = ((((int64_t(q.l) * B + q.b) * H + q.h) * S) + q.s) * D;
+    for (int x = threadIdx.x; x < dw; x += kAbsThreads) {   // channel pair x: entries red[e * dw + x]
+      uint32_t w = 0;
+      for (int e = 0; e < nrg; ++e) w = __vmaxu2(w, red[e * dw + x]);
+      const float a0 = lo_bf16(w), a1 = hi_bf16(w);
+      if (BITS == 8) {
+        float* t = static_cast<float*>(q.t ? va : ka) + t0;
+        t[2 * x] = a0;
+        t[2 * x + 1] = a1;
+      } else {
+        const uint32_t s0 = __float_as_uint(make_qscale<4>(a0).sc) >> 16, s1 = __float_as_uint(make_qscale<4>(a1).sc) >> 16;
+        reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(q.t ? va : ka) + t0)[x] = s0 | (s1 << 16);
+      }
+    }
+    __syncthreads();   // red is rewritten by the next unit
+  }
+}
+
+template <int BITS>
+__global__ void __launch_bounds__(kCodeThreads, 4) codes_kernel(
+    const uint4* __restrict__ k, const uint4* __restrict__ v, CompactParams p, const uint8_t* __restrict__ keep,
+    const int32_t* __restrict__ head_off, const int32_t* __restrict__ seg_off, const int64_t* __restrict__ layer_base,
+    void* __restrict__ kq, void* __restrict__ vq, const void* __restrict__ ka, const void* __restrict__ va) {
+  __shared__ int32_t chunk_prefix[kMaxGroupLH + 1];
+  __shared__ uint32_t keep_mask[kMaxGroupLH];
+  __shared__ int32_t warp_tot[kCodeThreads / 32];
+  const int S = p.sc.S, H = p.H, D = p.D, B = p.B;
+  const int nlh = p.nl * H;
+  const int lh0 = p.l0 * H;
+  for (int i = threadIdx.x; i < nlh; i += kCodeThreads) {
+    const uint8_t* kp = keep + int64_t(lh0 + i) * S;
+    uint32_t m = 0;
+    int32_t c = 0;
+    for (int s = 0; s < S; ++s)
+      if (kp[s]) {
+        m |= 1u << s;
+        c += (p.sc.n[s] + kCodeRows - 1) / kCodeRows;
+      }
+    keep_mask[i] = m;
+    chunk_prefix[i] = c;
+  }
+  __syncthreads();
+  block_exclusive_scan<kCodeThreads, kMaxGroupLH>(chunk_prefix, nlh, warp_tot);
+  const int32_t grand = chunk_prefix[nlh];
+  const int64_t units = int64_t(grand) * B * 2;     // (layer, batch, head, chunk) x {K, V}
+  const int cv_n = D / 8;
+  const int nrg = kCodeThreads / cv_n;
+  if (threadIdx.x >= nrg * cv_n) return;            // no block-wide barrier follows
+  const int cv = threadIdx.x % cv_n;
+  const int rg = threadIdx.x / cv_n;
+  for (int64_t g2 = blockIdx.x; g2 < units; g2 += gridDim.x) {
+    const int t = int(g2 & 1);
+    const int64_t g = g2 >> 1;
+    int la = 0, lz = p.nl;
+    while (lz - la > 1) {
+      const int mid = (la + lz) >> 1;
+      if (int64_t(chunk_prefix[mid * H]) * B <= g) la = mid; else lz = mid;
+    }
+    const int32_t c0 = chunk_prefix[la * H];
+    const int32_t C = chunk_prefix[(la + 1) * H] - c0;
+    const int64_t r = g - int64_t(c0) * B;
+    const int b = int(r / C);
+    const int32_t c = c0 + int32_t(r % C);
+    int lo = la * H, hi = (la + 1) * H;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (chunk_prefix[mid] <= c) lo = mid; else hi = mid;
+    }
+    int32_t j = c - chunk_prefix[lo];
+    const uint32_t m = keep_mask[lo];
+    int s = 0;
+    for (; s < S; ++s)
+      if (m >> s & 1u) {
+        const int32_t ch = (p.sc.n[s] + kCodeRows - 1) / kCodeRows;
+        if (j < ch) break;
+        j -= ch;
+      }
+    const int l = p.l0 + lo / H;
+    const int h = lo % H;
+    const int32_t r0 = j * kCodeRows;
+    const int32_t nrows = min(kCodeRows, p.sc.n[s] - r0);
+    // the 8 channels' scales of this block
+    const int64_t t0 = ((((int64_t(l) * B + b) * H + h) * S) + s) * D + cv * 8;
+    float sc[8], rc[8];
+    if (BITS == 8) {
+      const float* tab = static_cast<const float*>(t ? va : ka) + t0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const QScale qs = make_qscale<8>(tab[e]);
+        sc[e] = qs.sc;
+        rc[e] = qs.rc;
+      }
+    } else {
+      const uint4 w = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(t ? va : ka) + t0);
+      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        sc[2 * e] = lo_bf16(ww[e]);
+        sc[2 * e + 1] = hi_bf16(ww[e]);
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) rc[e] = (sc[e] >= 0x1p-100f && sc[e] <= 0x1p100f) ? __frcp_rn(sc[e]) : 0.f;
+    }
+    bool force = false;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) force |= sc[e] != 0.f && rc[e] == 0.f;
+    const uint4* src = (t ? v : k) +
+                       (int64_t(l) * p.layer_stride + ((int64_t(b) * H + h) * p.sc.T + p.sc.off[s] + r0) * D) / 8 + cv;
+    const int64_t R_l = (layer_base[l + 1] - layer_base[l]) / (int64_t(B) * D);
+    const int64_t e_first = layer_base[l] + (int64_t(b) * R_l + head_off[l * H + h] + seg_off[(l * H + h) * S + s] + r0) * D;
+    int32_t rr = rg;
+    if (BITS == 8) {
+      uint2* dst = reinterpret_cast<uint2*>(static_cast<int8_t*>(t ? vq : kq) + e_first) + cv;
+      for (; rr + 3 * nrg < nrows; rr += 4 * nrg) {
+        uint4 x[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[e] = __ldcs(src + (rr + e * nrg) * cv_n);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) __stcs(dst + (rr + e * nrg) * cv_n, codes8(x[e], sc, rc, force));
+      }
+      for (; rr < nrows; rr += nrg) __stcs(dst + rr * cv_n, codes8(__ldcs(src + rr * cv_n), sc, rc, force));
+    } else {
+      uint32_t* dst = static_cast<uint32_t*>(t ? vq : kq) + e_first / 8 + cv;
+      for (; rr + 3 * nrg < nrows; rr += 4 * nrg) {
+        uint4 x[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[e] = __ldcs(src + (rr + e * nrg) * cv_n);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) __stcs(dst + (rr + e * nrg) * cv_n, codes4x8(x[e], sc, rc, force));
+      }
+      for (; rr < nrows; rr += nrg) __stcs(dst + rr * cv_n, codes4x8(__ldcs(src + rr * cv_n), sc, rc, force));
+    }
+  }
 }
 
 // Dequantisation of one layer.  Unit = (batch, head, kept scale, chunk of at
@@ -643,13 +900,19 @@ struct DequantParams {
   int64_t R;               // rows per batch entry of the layer
 };
 
-__global__ void __launch_bounds__(kDeqThreads, 3) dequant_kernel(const uint2* __restrict__ kq,
-                                                              const uint2* __restrict__ vq,
-                                                              const float* __restrict__ ka,
-                                                              const float* __restrict__ va, DequantParams p,
+// BITS = 8: codes are uint2 per 8 elements, tables fp32 absmax (scale a / 127).
+// BITS = 4: codes are one uint32 word per 8 elements, tables bf16 scale bits.
+template <int BITS>
+__global__ void __launch_bounds__(kDeqThreads, 3) dequant_kernel(const void* __restrict__ kq_,
+                                                              const void* __restrict__ vq_,
+                                                              const void* __restrict__ ka_,
+                                                              const void* __restrict__ va_, DequantParams p,
                                                               const int32_t* __restrict__ head_off,
                                                               const int32_t* __restrict__ seg_off,
                                                               uint4* __restrict__ kc, uint4* __restrict__ vc) {
+  using CodeVec = typename std::conditional<BITS == 8, uint2, uint32_t>::type;
+  const CodeVec* __restrict__ kq = static_cast<const CodeVec*>(kq_);
+  const CodeVec* __restrict__ vq = static_cast<const CodeVec*>(vq_);
   __shared__ int32_t prefix[kDeqMaxH + 1];
   __shared__ uint32_t masks[kDeqMaxH];
   __shared__ int32_t warp_tot[kDeqThreads / 32];
@@ -678,7 +941,7 @@ __global__ void __launch_bounds__(kDeqThreads, 3) dequant_kernel(const uint2* __
   // bit flipped the byte is k + 128, placed as the low mantissa byte of
   // 1.5 * 2^23 (bits 0x4B400000) it reads 1.5 * 2^23 + k + 128, and one exact
   // subtraction leaves k.
-  auto expand = [](uint2 w, const float (&sc)[8]) {
+  auto expand8 = [](uint2 w, const float (&sc)[8]) {
     const uint2 wf = make_uint2(w.x ^ 0x80808080u, w.y ^ 0x80808080u);
     auto x = [](uint32_t u, int i) {
       return __fsub_rn(__uint_as_float(__byte_perm(u, 0x4B400000u, 0x7640u | uint32_t(i))), 12583040.0f);
@@ -689,6 +952,25 @@ __global__ void __launch_bounds__(kDeqThreads, 3) dequant_kernel(const uint2* __
     o.z = pack_bf16x2(__fmul_rn(x(wf.y, 0), sc[4]), __fmul_rn(x(wf.y, 1), sc[5]));
     o.w = pack_bf16x2(__fmul_rn(x(wf.y, 2), sc[6]), __fmul_rn(x(wf.y, 3), sc[7]));
     return o;
+  };
+  // A nibble n (code + 8) placed in the low mantissa bits of 1.5 * 2^23 reads
+  // 1.5 * 2^23 + n; subtracting 1.5 * 2^23 + 8 leaves the code exactly.  The
+  // product code * sc has at most 11 significant bits, so it is exact in fp32
+  // and the bf16 conversion rounds it once.
+  auto expand4 = [](uint32_t w, const float (&sc)[8]) {
+    auto x = [](uint32_t u, int shift) {
+      return __fsub_rn(__uint_as_float(0x4B400000u | ((u >> shift) & 0xFu)), 12582920.0f);
+    };
+    uint4 o;
+    o.x = pack_bf16x2(__fmul_rn(x(w, 0), sc[0]), __fmul_rn(x(w, 16), sc[1]));
+    o.y = pack_bf16x2(__fmul_rn(x(w, 4), sc[2]), __fmul_rn(x(w, 20), sc[3]));
+    o.z = pack_bf16x2(__fmul_rn(x(w, 8), sc[4]), __fmul_rn(x(w, 24), sc[5]));
+    o.w = pack_bf16x2(__fmul_rn(x(w, 12), sc[6]), __fmul_rn(x(w, 28), sc[7]));
+    return o;
+  };
+  auto expand = [&](CodeVec w, const float (&sc)[8]) {
+    if constexpr (BITS == 8) return expand8(w, sc);
+    else return expand4(w, sc);
   };
   // units in memory order (batch, head, kept chunk)
   for (int64_t g = blockIdx.x; g < units; g += gridDim.x) {
@@ -714,17 +996,30 @@ __global__ void __launch_bounds__(kDeqThreads, 3) dequant_kernel(const uint2* __
     const int64_t row0 = int64_t(b) * p.R + head_off[h] + seg_off[h * S + s] + r0;
     const int64_t arow = ((int64_t(b) * H + h) * S + s) * D + cv * 8;
     float sk[8], sv[8];
+    if constexpr (BITS == 8) {
+      const float* ka = static_cast<const float*>(ka_);
+      const float* va = static_cast<const float*>(va_);
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const float4 a = *reinterpret_cast<const float4*>(ka + arow + 4 * e);
-      const float4 bq = *reinterpret_cast<const float4*>(va + arow + 4 * e);
-      sk[4 * e] = a.x / 127.f; sk[4 * e + 1] = a.y / 127.f; sk[4 * e + 2] = a.z / 127.f; sk[4 * e + 3] = a.w / 127.f;
-      sv[4 * e] = bq.x / 127.f; sv[4 * e + 1] = bq.y / 127.f; sv[4 * e + 2] = bq.z / 127.f; sv[4 * e + 3] = bq.w / 127.f;
+      for (int e = 0; e < 2; ++e) {
+        const float4 a = *reinterpret_cast<const float4*>(ka + arow + 4 * e);
+        const float4 bq = *reinterpret_cast<const float4*>(va + arow + 4 * e);
+        sk[4 * e] = a.x / 127.f; sk[4 * e + 1] = a.y / 127.f; sk[4 * e + 2] = a.z / 127.f; sk[4 * e + 3] = a.w / 127.f;
+        sv[4 * e] = bq.x / 127.f; sv[4 * e + 1] = bq.y / 127.f; sv[4 * e + 2] = bq.z / 127.f; sv[4 * e + 3] = bq.w / 127.f;
+      }
+    } else {
+      const uint4 a = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(ka_) + arow);
+      const uint4 bq = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(va_) + arow);
+      const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {bq.x, bq.y, bq.z, bq.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        sk[2 * e] = lo_bf16(wa[e]); sk[2 * e + 1] = hi_bf16(wa[e]);
+        sv[2 * e] = lo_bf16(wb[e]); sv[2 * e + 1] = hi_bf16(wb[e]);
+      }
     }
     const int64_t e0 = row0 * cv_n + cv;
     int32_t r = rg;
     for (; r + 3 * nrg < nrows; r += 4 * nrg) {     // 4 rows' loads in flight, then the stores
-      uint2 ck[4], cw[4];
+      CodeVec ck[4], cw[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         ck[u] = __ldcs(kq + e0 + int64_t(r + u * nrg) * cv_n);
@@ -738,8 +1033,8 @@ __global__ void __launch_bounds__(kDeqThreads, 3) dequant_kernel(const uint2* __
     }
     for (; r < nrows; r += nrg) {
       const int64_t e = e0 + int64_t(r) * cv_n;
-      const uint2 ck = __ldcs(kq + e);
-      const uint2 cw = __ldcs(vq + e);
+      const CodeVec ck = __ldcs(kq + e);
+      const CodeVec cw = __ldcs(vq + e);
       kc[e] = expand(ck, sk);
       vc[e] = expand(cw, sv);
     }
@@ -750,11 +1045,11 @@ __global__ void __launch_bounds__(kDeqThreads, 3) dequant_kernel(const uint2* __
 
 using namespace vark;
 
-extern "C" int vark_quantize_kv_int8(const uint16_t* k, const uint16_t* v, int64_t layer_stride, int L, int B, int H,
-                                     int S, int D, const int32_t* sides, const uint8_t* keep,
-                                     const int32_t* head_off, const int32_t* seg_off, const int64_t* layer_base,
-                                     int8_t* kq, int8_t* vq, float* k_absmax, float* v_absmax, void* stream) {
-  if (!k || !v || !keep || !head_off || !seg_off || !layer_base || !kq || !vq || !k_absmax || !v_absmax)
+template <int BITS>
+static int quantize_kv(const uint16_t* k, const uint16_t* v, int64_t layer_stride, int L, int B, int H, int S, int D,
+                       const int32_t* sides, const uint8_t* keep, const int32_t* head_off, const int32_t* seg_off,
+                       const int64_t* layer_base, void* kq, void* vq, void* k_tab, void* v_tab, void* stream) {
+  if (!k || !v || !keep || !head_off || !seg_off || !layer_base || !kq || !vq || !k_tab || !v_tab)
     return VARK_E_ARG;
   QuantParams q;
   int rc = make_scale_table(S, sides, &q.sc);
@@ -765,14 +1060,13 @@ extern "C" int vark_quantize_kv_int8(const uint16_t* k, const uint16_t* v, int64
     if (int64_t(q.sc.n[s]) * (D / 8) >= INT32_MAX) return VARK_E_SHAPE;
   if (layer_stride < int64_t(B) * H * q.sc.T * D) return VARK_E_ARG;
   if (layer_stride % 8 != 0) return VARK_E_ALIGN;
-  if (!aligned16(k) || !aligned16(v) || !aligned16(kq) || !aligned16(vq) || !aligned16(k_absmax) ||
-      !aligned16(v_absmax))
+  if (!aligned16(k) || !aligned16(v) || !aligned16(kq) || !aligned16(vq) || !aligned16(k_tab) || !aligned16(v_tab))
     return VARK_E_ALIGN;
   if ((rc = check_device_sm100())) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int64_t nabs = int64_t(L) * B * H * S * D;
-  if (cudaMemsetAsync(k_absmax, 0, size_t(nabs) * 4, st) != cudaSuccess ||
-      cudaMemsetAsync(v_absmax, 0, size_t(nabs) * 4, st) != cudaSuccess)
+  const int64_t ntab = int64_t(L) * B * H * S * D * (BITS == 8 ? 4 : 2);
+  if (cudaMemsetAsync(k_tab, 0, size_t(ntab), st) != cudaSuccess ||
+      cudaMemsetAsync(v_tab, 0, size_t(ntab), st) != cudaSuccess)
     return VARK_E_CUDA;
   q.L = L; q.B = B; q.H = H; q.D = D; q.layer_stride = layer_stride;
   q.big_mask = 0;
@@ -788,34 +1082,53 @@ extern "C" int vark_quantize_kv_int8(const uint16_t* k, const uint16_t* v, int64
   cfg.blockDim = dim3(kQuantThreads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
-  if (cudaOccupancyMaxActiveClusters(&clusters, quant_kernel, &cfg) != cudaSuccess || clusters < 1) {
+  if (cudaOccupancyMaxActiveClusters(&clusters, quant_kernel<BITS>, &cfg) != cudaSuccess || clusters < 1) {
     cudaGetLastError();
     clusters = std::max(1, nsm / kQuantCluster);
   }
   const int layers_per_group = std::max(1, kQuantGroupLH / H);
+  if (kQuantTwoPass) {
+    CompactParams cp;
+    cp.sc = q.sc;
+    cp.L = L; cp.B = B; cp.H = H; cp.D = D; cp.layer_stride = layer_stride;
+    const int groups2 = std::max(1, std::min(layers_per_group, kMaxGroupLH / H));
+    for (int l0 = 0; l0 < L; l0 += groups2) {
+      q.l0 = cp.l0 = l0;
+      q.nl = cp.nl = std::min(groups2, L - l0);
+      absmax_kernel<BITS><<<nsm * 4, kAbsThreads, 0, st>>>(reinterpret_cast<const uint4*>(k),
+                                                           reinterpret_cast<const uint4*>(v), q, keep, k_tab, v_tab);
+      if (cudaGetLastError() != cudaSuccess) return VARK_E_CUDA;
+      codes_kernel<BITS><<<nsm * 4, kCodeThreads, 0, st>>>(
+          reinterpret_cast<const uint4*>(k), reinterpret_cast<const uint4*>(v), cp, keep, head_off, seg_off,
+          layer_base, kq, vq, k_tab, v_tab);
+      if (cudaGetLastError() != cudaSuccess) return VARK_E_CUDA;
+    }
+    return VARK_OK;
+  }
   for (int l0 = 0; l0 < L; l0 += layers_per_group) {
     q.l0 = l0;
     q.nl = std::min(layers_per_group, L - l0);
-    quant_kernel<<<clusters * kQuantCluster, kQuantThreads, 0, st>>>(
+    quant_kernel<BITS><<<clusters * kQuantCluster, kQuantThreads, 0, st>>>(
         reinterpret_cast<const uint4*>(k), reinterpret_cast<const uint4*>(v), q, keep, head_off, seg_off, layer_base,
-        kq, vq, k_absmax, v_absmax);
+        kq, vq, k_tab, v_tab);
     if (cudaGetLastError() != cudaSuccess) return VARK_E_CUDA;
   }
   return VARK_OK;
 }
 
-extern "C" int vark_dequantize_layer_int8(const int8_t* kq, const int8_t* vq, const float* k_absmax,
-                                          const float* v_absmax, int64_t kc_rows, int B, int H, int S, int D,
-                                          const int32_t* sides, const int32_t* head_off, const int32_t* seg_off,
-                                          uint16_t* kc, uint16_t* vc, void* stream) {
-  if (!kq || !vq || !k_absmax || !v_absmax || !head_off || !seg_off || !kc || !vc) return VARK_E_ARG;
+template <int BITS>
+static int dequantize_layer(const void* kq, const void* vq, const void* k_tab, const void* v_tab, int64_t kc_rows,
+                            int B, int H, int S, int D, const int32_t* sides, const int32_t* head_off,
+                            const int32_t* seg_off, uint16_t* kc, uint16_t* vc, void* stream) {
+  if (!kq || !vq || !k_tab || !v_tab || !head_off || !seg_off || !kc || !vc) return VARK_E_ARG;
   DequantParams p;
   int rc = make_scale_table(S, sides, &p.sc);
   if (rc) return rc;
   if (B < 1 || H < 1 || H > kDeqMaxH || D < 8 || D % 8 != 0 || D > 512 || kc_rows < 0 || kc_rows % B != 0)
     return VARK_E_SHAPE;
-  if (!aligned16(k_absmax) || !aligned16(v_absmax) || (reinterpret_cast<uintptr_t>(kq) & 7) ||
-      (reinterpret_cast<uintptr_t>(vq) & 7) || !aligned16(kc) || !aligned16(vc))
+  const uintptr_t code_align = BITS == 8 ? 7 : 3;
+  if (!aligned16(k_tab) || !aligned16(v_tab) || (reinterpret_cast<uintptr_t>(kq) & code_align) ||
+      (reinterpret_cast<uintptr_t>(vq) & code_align) || !aligned16(kc) || !aligned16(vc))
     return VARK_E_ALIGN;
   if ((rc = check_device_sm100())) return rc;
   if (kc_rows == 0) return VARK_OK;
@@ -823,8 +1136,39 @@ extern "C" int vark_dequantize_layer_int8(const int8_t* kq, const int8_t* vq, co
   int dev = 0, nsm = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  dequant_kernel<<<nsm * 3, kDeqThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-      reinterpret_cast<const uint2*>(kq), reinterpret_cast<const uint2*>(vq), k_absmax, v_absmax, p, head_off,
-      seg_off, reinterpret_cast<uint4*>(kc), reinterpret_cast<uint4*>(vc));
+  dequant_kernel<BITS><<<nsm * 3, kDeqThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      kq, vq, k_tab, v_tab, p, head_off, seg_off, reinterpret_cast<uint4*>(kc), reinterpret_cast<uint4*>(vc));
   return cudaGetLastError() == cudaSuccess ? VARK_OK : VARK_E_CUDA;
+}
+
+extern "C" int vark_quantize_kv_int8(const uint16_t* k, const uint16_t* v, int64_t layer_stride, int L, int B, int H,
+                                     int S, int D, const int32_t* sides, const uint8_t* keep,
+                                     const int32_t* head_off, const int32_t* seg_off, const int64_t* layer_base,
+                                     int8_t* kq, int8_t* vq, float* k_absmax, float* v_absmax, void* stream) {
+  return quantize_kv<8>(k, v, layer_stride, L, B, H, S, D, sides, keep, head_off, seg_off, layer_base, kq, vq,
+                        k_absmax, v_absmax, stream);
+}
+
+extern "C" int vark_quantize_kv_int4(const uint16_t* k, const uint16_t* v, int64_t layer_stride, int L, int B, int H,
+                                     int S, int D, const int32_t* sides, const uint8_t* keep,
+                                     const int32_t* head_off, const int32_t* seg_off, const int64_t* layer_base,
+                                     uint8_t* kq, uint8_t* vq, uint16_t* k_scale, uint16_t* v_scale, void* stream) {
+  return quantize_kv<4>(k, v, layer_stride, L, B, H, S, D, sides, keep, head_off, seg_off, layer_base, kq, vq,
+                        k_scale, v_scale, stream);
+}
+
+extern "C" int vark_dequantize_layer_int8(const int8_t* kq, const int8_t* vq, const float* k_absmax,
+                                          const float* v_absmax, int64_t kc_rows, int B, int H, int S, int D,
+                                          const int32_t* sides, const int32_t* head_off, const int32_t* seg_off,
+                                          uint16_t* kc, uint16_t* vc, void* stream) {
+  return dequantize_layer<8>(kq, vq, k_absmax, v_absmax, kc_rows, B, H, S, D, sides, head_off, seg_off, kc, vc,
+                             stream);
+}
+
+extern "C" int vark_dequantize_layer_int4(const uint8_t* kq, const uint8_t* vq, const uint16_t* k_scale,
+                                          const uint16_t* v_scale, int64_t kc_rows, int B, int H, int S, int D,
+                                          const int32_t* sides, const int32_t* head_off, const int32_t* seg_off,
+                                          uint16_t* kc, uint16_t* vc, void* stream) {
+  return dequantize_layer<4>(kq, vq, k_scale, v_scale, kc_rows, B, H, S, D, sides, head_off, seg_off, kc, vc,
+                             stream);
 }

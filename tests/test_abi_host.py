@@ -152,3 +152,119 @@ def test_generation_and_int8_calls_reject_bad_arguments_before_the_device():
     assert lib.vark_recompact_kv(p, p, p, p, p, 1, 1, 4, 7, 64, sides, 3, p, p, p, p, p, p, None) == -1
     q = ctypes.c_void_p(4096)
     assert lib.vark_recompact_kv(p, p, p, p, p, 1, 1, 4, 7, 64, sides, 8, p, p, p, p, q, q, None) == -1
+
+
+def test_size_limits_are_status_codes():
+    """Shapes whose arithmetic would overflow, or whose calibration tiles would
+    not fit in shared memory, are refused before any array is read or any
+    device call is made."""
+    lib = vark.library()
+    p = ctypes.c_void_p(16)
+    # calibration at D = 128: 30 scales fit the shared memory, 31 do not (D = 64: 32 fit)
+    s31 = (ctypes.c_int32 * 31)(*([1] * 31))
+    s30 = (ctypes.c_int32 * 30)(*([1] * 30))
+    s32 = (ctypes.c_int32 * 32)(*([1] * 32))
+    assert lib.vark_scas_accumulate(p, p, p, 1, 4, 128, 31, s31, p, None, p, None, p, None) == -2
+    assert lib.vark_scas_accumulate(p, p, p, 1, 4, 128, 30, s30, p, None, p, None, p, None) in (-7, -5, 0)
+    assert lib.vark_scas_accumulate(p, p, p, 1, 4, 64, 32, s32, p, None, p, None, p, None) in (-7, -5, 0)
+    # schedule budget arithmetic: F = L * H * T tokens with F * 10000 < 2^63.  32 scales of side
+    # 4096 give T = 2^29; L * H = 2^20 makes F = 2^49 (fits), 2^21 makes 2^50 > 9.2e14.  The
+    # arrays passed are tiny: a refused shape must not read them.
+    big = (ctypes.c_int32 * 32)(*([4096] * 32))
+    tiny = np.zeros(8)
+    keep = np.zeros(8, dtype=np.uint8)
+    assert lib.vark_build_schedule(tiny.ctypes.data, 1 << 11, 1 << 10, 32, big, 5000, 2, keep.ctypes.data) == -2
+    assert lib.vark_rank_stability(tiny.ctypes.data, tiny.ctypes.data, 1 << 11, 1 << 10, 32, big, 5000, 2,
+                                   ctypes.byref(ctypes.c_double()), ctypes.byref(ctypes.c_double())) == -2
+    pre = np.zeros(32, dtype=np.int32)
+    assert lib.vark_build_early_pruning_schedule(tiny.ctypes.data, 1 << 11, 1 << 10, 32, big, 5000, 2,
+                                                 pre.ctypes.data, keep.ctypes.data) == -2
+    out = np.zeros(8, dtype=np.int64)
+    assert lib.vark_cache_size_after_layer(keep.ctypes.data, 1 << 16, 1 << 10, 32, big, 1 << 10, 128,
+                                           out.ctypes.data) == -2
+    # the same builder at a small size still works
+    sc = np.random.default_rng(3).uniform(size=(2, 3, 7))
+    assert np.array_equal(vark.vark_build_schedule(sc, SIDES_TINY, 5000, 2), oracle.build_schedule(sc, SIDES_TINY,
+                                                                                                   5000, 2))
+
+
+def test_binding_refuses_mismatched_tensor_sizes():
+    """Every wrapper compares its tensors with the shape it hands to the C call
+    and raises ValueError before a pointer is taken (CPU tensors here: the size
+    check comes first, so nothing reaches the library)."""
+    import torch
+    sides = SIDES_TINY
+    S, T, D, B, H = 7, 155, 64, 2, 4
+    bf = torch.bfloat16
+    f32 = torch.float32
+    i32 = torch.int32
+    q = torch.zeros((B, H, T, D), dtype=bf)
+    st = torch.zeros(1, dtype=i32)
+    tau, bias, mass = torch.zeros(H), torch.zeros(H, S), torch.zeros(H, S, S)
+    good = dict(q=q, k=q, v=q, sides=sides, tau=tau, bias=bias, mass=mass, out=q, dev_status=st)
+    for key, bad in (("q", torch.zeros((B, H, T - 1, D), dtype=bf)), ("k", torch.zeros((B, H, T, 32), dtype=bf)),
+                     ("v", torch.zeros((B + 1, H, T, D), dtype=bf)), ("out", torch.zeros((B, H, T, D + 8), dtype=bf)),
+                     ("tau", torch.zeros(H - 1)), ("bias", torch.zeros(H, S - 1)), ("mass", torch.zeros(H, S, S - 1))):
+        with pytest.raises(ValueError):
+            vark.vark_scas_accumulate(**{**good, key: bad})
+    with pytest.raises(TypeError):          # sizes right: the device check is what refuses a CPU tensor
+        vark.vark_scas_accumulate(**good)
+    L = 2
+    keep = torch.ones((L, H, S), dtype=torch.uint8)
+    tabs = dict(head_off=torch.zeros(L, H, dtype=i32), seg_off=torch.zeros(L, H, S, dtype=i32),
+                past_len=torch.zeros(L, H, S, dtype=i32), layer_base=torch.zeros(L + 1, dtype=torch.int64))
+    for key in tabs:
+        bad = torch.zeros(tabs[key].numel() + 1, dtype=tabs[key].dtype)
+        with pytest.raises(ValueError):
+            vark.vark_build_offsets(keep, sides, B, D, **{**tabs, key: bad})
+    kd = torch.zeros((L, B, H, T, D), dtype=bf)
+    comp = dict(k=kd, v=kd, layer_stride=B * H * T * D, L=L, B=B, H=H, sides=sides, D=D, keep=keep,
+                head_off=tabs["head_off"], seg_off=tabs["seg_off"], layer_base=tabs["layer_base"], kc=kd, vc=kd)
+    for key, bad in (("k", kd[:1]), ("layer_stride", B * H * T * D - 8), ("keep", keep[:1]),
+                     ("seg_off", tabs["seg_off"][:1])):
+        with pytest.raises(ValueError):
+            vark.vark_compact_kv(**{**comp, key: bad})
+    # pruned attention: one layer, every query scale
+    pr = dict(q=q, kc=torch.zeros(B * 10 * D, dtype=bf), vc=torch.zeros(B * 10 * D, dtype=bf), kc_rows=B * 10,
+              k_dense=q, v_dense=q, sides=sides, query_scale=-1, head_off=torch.zeros(H, dtype=i32),
+              seg_off=torch.zeros(H, S, dtype=i32), past_len=torch.zeros(H, S, dtype=i32), tau=tau, bias=bias,
+              out=q, dev_status=st)
+    for key, bad in (("q", torch.zeros((B, H, 64, D), dtype=bf)), ("kc", torch.zeros(B * 10 * D - 1, dtype=bf)),
+                     ("kc_rows", B * 10 + 1), ("out", q[:1]), ("head_off", torch.zeros(H + 1, dtype=i32)),
+                     ("past_len", torch.zeros(H, dtype=i32)), ("query_scale", S)):
+        with pytest.raises(ValueError):
+            vark.vark_pruned_attention(**{**pr, key: bad})
+    q6 = torch.zeros((B, H, 64, D), dtype=bf)
+    with pytest.raises(TypeError):          # query scale 6 (64 rows): sizes right
+        vark.vark_pruned_attention(**{**pr, "q": q6, "out": q6, "query_scale": 6})
+    step = {**pr, "q": q6, "out": q6, "scale": 6}
+    step.pop("query_scale")
+    step["k_local"] = step.pop("k_dense")
+    step["v_local"] = step.pop("v_dense")
+    with pytest.raises(ValueError):         # k_local must hold the scale's rows only
+        vark.vark_pruned_attention_step(**step)
+    with pytest.raises(ValueError):
+        vark.vark_dequantize_layer_int8(torch.zeros(10, dtype=torch.int8), torch.zeros(10, dtype=torch.int8),
+                                        torch.zeros(B * H * S * D), torch.zeros(B * H * S * D), 2, 1, H, sides, D,
+                                        torch.zeros(H, dtype=i32), torch.zeros(H, S, dtype=i32),
+                                        torch.zeros(2 * D, dtype=bf), torch.zeros(2 * D, dtype=bf))
+
+
+def test_int4_calls_reject_bad_arguments_before_the_device():
+    lib = vark.library()
+    sides = (ctypes.c_int32 * 7)(*SIDES_TINY)
+    p = ctypes.c_void_p(16)
+    odd = ctypes.c_void_p(24)           # 8-byte but not 16-byte aligned
+    two = ctypes.c_void_p(18)           # 2-byte aligned only
+    # quantising compaction: k, v, layer_stride, L, B, H, S, D, sides, keep, head_off, seg_off, layer_base, kq, vq, ks, vs
+    assert lib.vark_quantize_kv_int4(None, p, 1 << 20, 1, 1, 4, 7, 64, sides, p, p, p, p, p, p, p, p, None) == -1
+    assert lib.vark_quantize_kv_int4(p, p, 1 << 20, 1, 1, 4, 7, 60, sides, p, p, p, p, p, p, p, p, None) == -2
+    assert lib.vark_quantize_kv_int4(p, p, 100, 1, 1, 4, 7, 64, sides, p, p, p, p, p, p, p, p, None) == -1
+    assert lib.vark_quantize_kv_int4(p, p, 1 << 20, 1, 1, 4, 7, 64, sides, p, p, p, p, odd, p, p, p, None) == -3
+    assert lib.vark_quantize_kv_int4(p, p, 1 << 20, 1, 1, 4, 7, 64, sides, p, p, p, p, p, p, odd, p, None) == -3
+    # dequantisation: kq, vq, ks, vs, kc_rows, B, H, S, D, sides, head_off, seg_off, kc, vc (codes 4-byte aligned)
+    assert lib.vark_dequantize_layer_int4(None, p, p, p, 8, 1, 4, 7, 64, sides, p, p, p, p, None) == -1
+    assert lib.vark_dequantize_layer_int4(p, p, p, p, 9, 2, 4, 7, 64, sides, p, p, p, p, None) == -2
+    assert lib.vark_dequantize_layer_int4(two, p, p, p, 8, 1, 4, 7, 64, sides, p, p, p, p, None) == -3
+    assert lib.vark_dequantize_layer_int4(ctypes.c_void_p(20), p, p, p, 8, 1, 4, 7, 64, sides, p, p, p, p,
+                                          None) in (-7, -5, 0)

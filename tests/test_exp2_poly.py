@@ -1,7 +1,12 @@
-"""The FMA-pipe 2^x used for part of the softmax exponentials: the kernel
-header's coefficients and reduction, evaluated step by step in fp32 on the
-CPU, stay within the stated relative error of 2^x over the whole input range
-the kernels feed it (clamped at -125, so results stay normal fp32)."""
+"""The FMA-pipe 2^x used for part of the softmax exponentials.
+
+* The kernel header's coefficients are the degree-3 minimax polynomial of 2^f
+  on [-1/2, 1/2] in relative error, rounded to fp32: the Remez exchange below
+  re-derives them from that definition (Cody-Waite reduction x = n + f with
+  n = round(x), so 2^x = 2^n * P(f)).
+* The header's reduction and coefficients, evaluated step by step in fp32 on
+  the CPU, stay within the stated relative error of 2^x over the whole input
+  range the kernels feed it (clamped at -125, so results stay normal fp32)."""
 import os
 import re
 
@@ -17,6 +22,36 @@ def _coefficients():
     body = body[:body.index("\n}\n")]
     vals = dict(re.findall(r"(c[0-3]) = ([0-9.eE+-]+)f", body))
     return [np.float32(vals[f"c{i}"]) for i in range(4)]
+
+
+def _remez_exp2(deg=3, a=-0.5, b=0.5, iters=30):
+    """Minimax polynomial of 2^f on [a, b] in relative error: solve for
+    equioscillating relative error E at deg + 2 reference points, move the
+    references to the extrema of the new error curve, repeat."""
+    n = deg + 2
+    x = np.cos(np.pi * np.arange(n) / (n - 1))[::-1] * (b - a) / 2 + (a + b) / 2
+    grid = np.linspace(a, b, 20001)
+    for _ in range(iters):
+        A = np.zeros((n, n))
+        for i in range(n):
+            A[i, :deg + 1] = x[i] ** np.arange(deg + 1)
+            A[i, deg + 1] = (-1) ** i * 2.0 ** x[i]
+        sol = np.linalg.solve(A, 2.0 ** x)
+        c = sol[:deg + 1]
+        err = (np.polyval(c[::-1], grid) - 2.0 ** grid) / 2.0 ** grid
+        idx = [0] + [i for i in range(1, len(grid) - 1)
+                     if (err[i] - err[i - 1]) * (err[i + 1] - err[i]) < 0] + [len(grid) - 1]
+        if len(idx) != n:
+            break
+        x = grid[idx]
+    return c, float(np.abs(err).max())
+
+
+def test_coefficients_are_the_remez_fit():
+    c, e = _remez_exp2()
+    assert 7.0e-5 < e < 8.0e-5           # the minimax error of degree 3 on [-1/2, 1/2]
+    hdr = np.array(_coefficients(), dtype=np.float64)
+    np.testing.assert_allclose(hdr, c.astype(np.float32).astype(np.float64), rtol=2e-6)
 
 
 def _device_exp2(x):

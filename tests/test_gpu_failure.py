@@ -68,4 +68,4 @@ def test_withheld_key_tile_times_out_and_context_stays_usable(monkeypatch):
     assert status == 0
     O_ref, m_ref = oracle.block_causal_attention(*(f64(b) for b in bits), tiny, tau.astype(np.float64), None)
     assert np.abs(f64(bits_of(out)) - O_ref).max() <= 2e-2
-    np.testing.assert_allclose(mass.cpu().numpy(), oracle.scas_mass(m_ref, tiny), rtol=1e-3, atol=1e-6)
+    np.testing.assert_allclose(mass.cpu().numpy(), oracle.scas_mass(m_ref, tiny), rtol=1e-3)

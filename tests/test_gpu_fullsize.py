@@ -68,7 +68,7 @@ def _pipeline(wname):
         bias = synth.gen_bias(synth.layer_seed(w, l), H, g.S) if w.with_bias else None
         out = pruned_layer(q, kc, vc, kd[l], vd[l], tab, l, sides, -1, torch.from_numpy(tau).cuda(),
                            None if bias is None else torch.from_numpy(bias).cuda())
-        for _ in range(2):
+        for _ in range(4):
             b, h = int(rng.integers(B)), int(rng.integers(H))
             kf = f64(synth.rows_bf16_bits(kkey, shape, (l, b, h), 0, T))
             vf = f64(synth.rows_bf16_bits(vkey, shape, (l, b, h), 0, T))
@@ -117,7 +117,7 @@ def test_larger_model_calibration_launch_full_size():
             _, m = oracle.attention_rows(qb[g.off[kk]:g.L[kk]], kb, vb, sides, kk, float(tau[h]),
                                          bias[h].astype(np.float64))
             acc[:, kk] += m.sum(axis=0) / (Bc * g.n[kk])
-    np.testing.assert_allclose(M[h, :, :8], acc, rtol=1e-3, atol=1e-6)
+    np.testing.assert_allclose(M[h, :, :8], acc, rtol=1e-3)
     b, kk = Bc - 1, 12
     rows = np.array([0, 127, 128, 4095])
     kb, vb = (f64(synth.rows_bf16_bits(key, shape, (b, h), 0, T)) for key in keys[1:])

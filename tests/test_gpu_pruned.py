@@ -98,6 +98,25 @@ def test_pruned_1024_sampled_rows_all_scales():
                 assert np.abs(O_gpu[b, h, g.off[kk] + rows] - o_ref).max() <= O_ATOL, (b, h, kk)
 
 
+def test_pruned_1024_ten_heads_full():
+    """1024^2 scales, 10 heads (the launch interleaves heads in groups of 8, so
+    the last group is partial), ragged keep with a head that keeps nothing
+    and one that keeps everything, bias: every output element of every scale
+    against the oracle."""
+    sides = SIDES_1024
+    g = oracle.ScaleGeometry(sides)
+    B, H, D = 1, 10, 128
+    qb, kb, vb, tau, bias = _layer_inputs(sides, B, H, D, 15, True)
+    keep = np.random.default_rng(15).integers(0, 2, size=(H, g.S)).astype(np.uint8)
+    keep[:, :2] = 1
+    keep[3, :] = 0
+    keep[7, :] = 1
+    O_gpu = _run(qb, kb, vb, keep, sides, tau, bias, -1)
+    O_ref = oracle.pruned_attention(f64(qb), f64(kb), f64(vb), keep, sides, tau.astype(np.float64),
+                                    bias.astype(np.float64))
+    assert np.abs(O_gpu - O_ref).max() <= O_ATOL
+
+
 def oatt_rows(q_rows, kf, vf, keep_h, sides, kk, tau_h, bias_h):
     from oracle.attention import pruned_attention_rows
     return pruned_attention_rows(q_rows, kf, vf, keep_h, sides, kk, float(tau_h),
@@ -105,7 +124,7 @@ def oatt_rows(q_rows, kf, vf, keep_h, sides, kk, tau_h, bias_h):
 
 
 @pytest.mark.parametrize("budget_bp", [10000, 2000, 1000, 400])
-@pytest.mark.parametrize("B", [1, 4, 32])
+@pytest.mark.parametrize("B", [1, 4, 16, 32])
 def test_final_scale_sweep_sampled(budget_bp, B):
     """The 64x64 scale's 4,096 queries against the 10,521-token cache with
     seed-random retained sets per head (final-scale sweep), inputs made on the
@@ -124,8 +143,8 @@ def test_final_scale_sweep_sampled(budget_bp, B):
     kc, vc = compact(kd[None], vd[None], tab, sides)
     out = pruned_layer(q, kc, vc, kd, vd, tab, 0, sides, kq, torch.from_numpy(tau).cuda(), None)
     rng = np.random.default_rng(budget_bp + B)
-    for _ in range(3):
-        b, h = int(rng.integers(B)), int(rng.integers(H))
+    pairs = {(B - 1, H - 1)} | {(int(rng.integers(B)), int(rng.integers(H))) for _ in range(5)}
+    for b, h in sorted(pairs):
         rows = np.unique(np.concatenate([[0, 127, 128, g.n[kq] - 1], rng.integers(0, g.n[kq], size=4)]))
         kf = f64(synth.rows_bf16_bits(keys[1], (B, H, T, D), (b, h), 0, T))
         vf = f64(synth.rows_bf16_bits(keys[2], (B, H, T, D), (b, h), 0, T))

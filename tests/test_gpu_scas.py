@@ -13,8 +13,7 @@ from tests.helpers import bits_of, check_status, dev_bf16, f64, status_word
 pytestmark = pytest.mark.gpu
 
 O_ATOL = 2e-2
-MASS_RTOL = 1e-3
-MASS_ATOL = 1e-6
+MASS_RTOL = 1e-3   # relative only: entries s > k are exactly 0 on both sides
 
 
 def _calib_inputs(sides, B, H, D, seed, with_bias):
@@ -48,39 +47,88 @@ def test_scas_tiny_full_parity(with_bias):
                                                 None if bias is None else bias.astype(np.float64))
     M_ref = oracle.scas_mass(mass, sides)
     assert np.abs(O_gpu - O_ref).max() <= O_ATOL
-    np.testing.assert_allclose(M_gpu, M_ref, rtol=MASS_RTOL, atol=MASS_ATOL)
+    np.testing.assert_allclose(M_gpu, M_ref, rtol=MASS_RTOL)
     # S-CAS through the library's host finaliser vs the oracle's
     sc_gpu = vark.vark_scas_finalize(M_gpu.astype(np.float32)[None])
     sc_ref = oracle.scas_from_mass(M_ref[None])
-    np.testing.assert_allclose(sc_gpu, sc_ref, rtol=MASS_RTOL, atol=MASS_ATOL)
+    np.testing.assert_allclose(sc_gpu, sc_ref, rtol=MASS_RTOL)
 
 
-def test_scas_tiny_schedule_parity_when_gaps_are_clear():
-    """GPU S-CAS -> host schedule equals the oracle's whenever neighbouring
-    oracle S-CAS values differ by more than 1e-4."""
+def _gaps_clear_along_drop_order(sc_ref, sc_gpu, keep_ref, n_sinks, gap=1e-4):
+    """The schedule-parity condition where it decides the result.  The greedy
+    walk drops candidates in ascending (S-CAS, l, h, s) order and stops at the
+    first prefix that meets the budget, so the order of every candidate up to
+    and including the first retained one matters (a near-tie anywhere in that
+    prefix can change where the walk stops).  Along that prefix two neighbours
+    must be more than `gap` apart, or an exact tie on BOTH sides (e.g. the last
+    scale, which no later scale reads, scores exactly 0): exact ties are broken
+    by index identically by both builders."""
+    L, H, S = sc_ref.shape
+    cand = sorted((float(sc_ref[l, h, s]), l, h, s) for l in range(L) for h in range(H) for s in range(n_sinks, S))
+    n_drop = int((keep_ref[:, :, n_sinks:] == 0).sum())
+    prefix = cand[:n_drop + 1]
+    for (a, *ia), (b, *ib) in zip(prefix, prefix[1:]):
+        if a == b:
+            if sc_gpu[tuple(ia)] != sc_gpu[tuple(ib)]:
+                return False
+        elif b - a <= gap:
+            return False
+    return True
+
+
+def _schedule_parity(M_gpu, M_ref, sides, budgets, n_sinks=2):
+    sc_gpu = vark.vark_scas_finalize(np.stack(M_gpu).astype(np.float32))
+    sc_ref = oracle.scas_from_mass(np.stack(M_ref))
+    np.testing.assert_allclose(sc_gpu, sc_ref, rtol=MASS_RTOL)
+    checked = 0
+    for budget in budgets:
+        keep_ref = oracle.build_schedule(sc_ref, sides, budget, n_sinks)
+        keep_gpu = vark.vark_build_schedule(sc_gpu, sides, budget, n_sinks)
+        # the builder itself is exact on the same input
+        assert np.array_equal(vark.vark_build_schedule(sc_ref, sides, budget, n_sinks), keep_ref)
+        # the seeds are chosen so that the condition holds: the comparison runs
+        assert _gaps_clear_along_drop_order(sc_ref, sc_gpu, keep_ref, n_sinks), budget
+        assert int((keep_ref[:, :, n_sinks:] == 0).sum()) > 0
+        assert np.array_equal(keep_gpu, keep_ref), budget
+        checked += 1
+    assert checked == len(budgets)
+
+
+def test_scas_tiny_schedule_parity():
+    """GPU S-CAS -> host schedule equals the oracle's schedule bit for bit
+    (3 layers x 4 heads, tiny scales, budgets from 55% down to 20%: every
+    budget drops pairs beyond the last scale's structural zeros)."""
     sides = SIDES_TINY
     L, H, B = 3, 4, 4
     M_gpu, M_ref = [], []
     for l in range(L):
-        bits, tau, _ = _calib_inputs(sides, B, H, 64, 10 + l, False)
+        bits, tau, _ = _calib_inputs(sides, B, H, 64, 37 + l, False)
         Mg, _ = _gpu_calib(bits, sides, tau, None, want_out=False)
         q, k, v = (f64(b) for b in bits)
         _, mass = oracle.block_causal_attention(q, k, v, sides, tau.astype(np.float64), None)
         M_gpu.append(Mg)
         M_ref.append(oracle.scas_mass(mass, sides))
-    sc_gpu = vark.vark_scas_finalize(np.stack(M_gpu).astype(np.float32))
-    sc_ref = oracle.scas_from_mass(np.stack(M_ref))
-    vals = np.sort(sc_ref[:, :, 2:].ravel())
-    checked = 0
-    for budget in (8000, 5000, 3000):
-        keep_ref = oracle.build_schedule(sc_ref, sides, budget, 2)
-        keep_gpu = vark.vark_build_schedule(sc_gpu, sides, budget, 2)
-        if np.all(np.diff(vals) > 1e-4):
-            assert np.array_equal(keep_gpu, keep_ref)
-            checked += 1
-        # the builder itself is exact on the same input
-        assert np.array_equal(vark.vark_build_schedule(sc_ref, sides, budget, 2), keep_ref)
-    assert checked in (0, 3)
+    _schedule_parity(M_gpu, M_ref, sides, (5500, 5000, 4000, 3000, 2000))
+
+
+@pytest.mark.slow
+def test_scas_1024_schedule_parity():
+    """1024^2 scales with bias, 2 layers x 4 heads x 2 calibration seeds: GPU
+    calibration (with O, as in the benchmark step) -> S-CAS -> schedule at 10%
+    and 4% equals the oracle's; the mass matches in full."""
+    sides = SIDES_1024
+    L, H, B = 2, 4, 2
+    M_gpu, M_ref = [], []
+    for l in range(L):
+        bits, tau, bias = _calib_inputs(sides, B, H, 128, 8 + l, True)
+        Mg, _ = _gpu_calib(bits, sides, tau, bias, want_out=True)
+        q, k, v = (f64(b) for b in bits)
+        _, mass = oracle.block_causal_attention(q, k, v, sides, tau.astype(np.float64), bias.astype(np.float64))
+        Mr = oracle.scas_mass(mass, sides)
+        np.testing.assert_allclose(Mg, Mr, rtol=MASS_RTOL)
+        M_gpu.append(Mg)
+        M_ref.append(Mr)
+    _schedule_parity(M_gpu, M_ref, sides, (1000, 400))
 
 
 def test_scas_1024_two_seeds_two_heads_full_parity():
@@ -91,7 +139,7 @@ def test_scas_1024_two_seeds_two_heads_full_parity():
     O_ref, mass = oracle.block_causal_attention(q, k, v, sides, tau.astype(np.float64), bias.astype(np.float64))
     M_ref = oracle.scas_mass(mass, sides)
     assert np.abs(O_gpu - O_ref).max() <= O_ATOL
-    np.testing.assert_allclose(M_gpu, M_ref, rtol=MASS_RTOL, atol=MASS_ATOL)
+    np.testing.assert_allclose(M_gpu, M_ref, rtol=MASS_RTOL)
 
 
 @pytest.mark.parametrize("sides,B,H,D", [(SIDES_TINY, 4, 4, 64), (SIDES_1024, 2, 2, 128), (SIDES_1024, 3, 1, 64)])
@@ -105,8 +153,8 @@ def test_scas_without_output_matches_oracle(sides, B, H, D):
     q, k, v = (f64(b) for b in bits)
     _, mass = oracle.block_causal_attention(q, k, v, sides, tau.astype(np.float64), bias.astype(np.float64))
     M_ref = oracle.scas_mass(mass, sides)
-    np.testing.assert_allclose(M_noo, M_ref, rtol=MASS_RTOL, atol=MASS_ATOL)
-    np.testing.assert_allclose(M_noo, M_o, rtol=1e-5, atol=1e-7)
+    np.testing.assert_allclose(M_noo, M_ref, rtol=MASS_RTOL)
+    np.testing.assert_allclose(M_noo, M_o, rtol=MASS_RTOL)
     S = len(sides)
     for kk in range(S):
         np.testing.assert_allclose(M_noo[:, :kk + 1, kk].sum(axis=1), 1.0, atol=1e-4)
@@ -115,8 +163,9 @@ def test_scas_without_output_matches_oracle(sides, B, H, D):
 @pytest.mark.slow
 def test_scas_calibration_full_size_sampled():
     """16 seeds x 16 heads at 1024^2, inputs made on the device: mass sums to
-    one per (h, k); M for scales <= 8 of two heads and sampled output rows of
-    every scale against the oracle."""
+    one per (h, k); M of one head for every query scale and of another for the
+    scales <= 8, and sampled output rows of several scales, against the
+    oracle."""
     w = synth.WORKLOADS["calib_1024"]
     sides, H, D, B = w.sides, w.heads, w.head_dim, w.n_seeds
     T = synth.n_tokens(sides)
@@ -137,18 +186,20 @@ def test_scas_calibration_full_size_sampled():
         np.testing.assert_allclose(M[:, :kk + 1, kk].sum(axis=1), 1.0, atol=1e-4)
         assert np.all(M[:, kk + 1:, kk] == 0)
     shape = (B, H, T, D)
-    for h in (0, 11):
-        Lk = g.L[8]
-        acc = np.zeros((S, 9))
+    # head 11: M for every query scale (scales 9-12 carry ~98% of the work);
+    # head 0: the scales <= 8
+    for h, n_k in ((11, S), (0, 9)):
+        Lk = g.L[n_k - 1]
+        acc = np.zeros((S, n_k))
         for b in range(B):
             kb = f64(synth.rows_bf16_bits(keys[1], shape, (b, h), 0, Lk))
             vb = f64(synth.rows_bf16_bits(keys[2], shape, (b, h), 0, Lk))
             qb = f64(synth.rows_bf16_bits(keys[0], shape, (b, h), 0, Lk))
-            for kk in range(9):
+            for kk in range(n_k):
                 r0, r1 = g.off[kk], g.L[kk]
                 _, m = oracle.attention_rows(qb[r0:r1], kb, vb, sides, kk, float(tau[h]), bias[h].astype(np.float64))
                 acc[:, kk] += m.sum(axis=0) / (B * g.n[kk])
-        np.testing.assert_allclose(M[h, :, :9], acc, rtol=MASS_RTOL, atol=MASS_ATOL)
+        np.testing.assert_allclose(M[h, :, :n_k], acc, rtol=MASS_RTOL)
     rng = np.random.default_rng(0)
     for kk in (0, 5, 9, 12):
         b, h = int(rng.integers(B)), int(rng.integers(H))

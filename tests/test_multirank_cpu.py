@@ -1,6 +1,8 @@
 """N > 1 host logic of the benchmark on CPU with gloo: every rank runs its own
-replica; timings are reduced max-over-ranks and work sum-over-ranks; the
-reference (oracle) arm runs on rank 0 only and the other ranks exit at once."""
+replica on inputs drawn from its own seed (checked by gathering each rank's
+first generated values); timings are reduced max-over-ranks and work
+sum-over-ranks; the reference (oracle) arm runs on rank 0 only and the other
+ranks exit at once."""
 import os
 import subprocess
 import sys
@@ -23,9 +25,16 @@ def _worker(rank, world, port, q):
     dev = torch.device("cpu")
     mx = bench.reduce_over_ranks(1.5 + rank, "max", world, dev)
     sm = bench.reduce_over_ranks(10.0 * (rank + 1), "sum", world, dev)
+    # each replica's inputs: the first values of its calibration q, made by the
+    # benchmark's own generator from the rank's seed
+    w = bench.synth.WORKLOADS[bench.WORKLOAD]
+    mine = bench.randn_bf16((1, 64), bench.replica_seed(w, rank) + 1, dev).float()
+    gathered = [torch.empty_like(mine) for _ in range(world)]
+    dist.all_gather(gathered, mine)
+    distinct = all(not torch.equal(gathered[i], gathered[j]) for i in range(world) for j in range(i + 1, world))
     dist.barrier()
     dist.destroy_process_group()
-    q.put((rank, mx, sm))
+    q.put((rank, mx, sm, distinct))
 
 
 @pytest.mark.parametrize("world", [2])
@@ -40,9 +49,10 @@ def test_timing_reductions_over_gloo_ranks(world):
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    for rank, mx, sm in res:
+    for rank, mx, sm, distinct in res:
         assert mx == 1.5 + (world - 1)
         assert sm == 10.0 * world * (world + 1) / 2
+        assert distinct            # replicas are independent: no two ranks draw the same inputs
 
 
 def test_reference_arm_nonzero_rank_exits_without_work():
