@@ -97,8 +97,22 @@ struct Params {
 // keys: the softmax stores a chunk as soon as its exponentials are done and
 // the MMA thread issues that chunk's share of PV_X at once, so PV_X overlaps
 // the rest of the softmax instead of following it.
-constexpr int kPChunks = 4;
-constexpr int kChunkKeys = kBlockN / kPChunks;   // 32 keys = 16 TMEM columns of bf16 pairs
+// Per tile, kPChunks barrier slots; a kernel uses PChunks<...>::kCount of them.
+// (The slot count is kept at the largest kCount: the barrier block and the
+// shared-memory layout after it then match the one-chunk kernel's.)
+// Calibration with O (whose softmax still has the mass partials to add after
+// P is stored) gains from 2 chunks of 64 keys, each signalled per warp
+// (967 vs 947 TFLOP/s in an interleaved same-box A/B; 4 chunks: 900); pruned
+// attention and S-CAS-only calibration measured best with one P store
+// signalled by every thread (2-7% and 6% ahead of 2 chunks).
+constexpr int kPChunks = 2;
+template <bool MASS, bool WITH_O>
+struct PChunks {
+  static constexpr int kCount = (MASS && WITH_O) ? 2 : 1;
+  static constexpr int kKeys = kBlockN / kCount;          // keys per chunk
+  static constexpr bool kPerWarp = kCount > 1;             // one arrival per warp (else per thread)
+  static constexpr int kArrivals = kPerWarp ? kBlockM / 32 : kBlockM;
+};
 
 enum Bar {
   kBarQ = 0,
@@ -108,10 +122,17 @@ enum Bar {
   kBarVEmpty = 7,     // [2]
   kBarSFull = 9,      // [tile]
   kBarPFull = 11,     // [tile][kPChunks]; without O, chunk 0 = "S_X read"
-  kBarODone = 19,     // [tile]
-  kBarDrain = 21,
-  kNumBars = 22
+  kBarODone = 15,     // [tile]
+  kBarDrain = 17,
+  kNumBars = 18
 };
+
+// Store one P chunk (kKeys / 2 columns of bf16 pairs) into TMEM.
+VARK_DEV void tmem_st_chunk(uint32_t taddr, const uint32_t (&r)[32]) { tmem_st32(taddr, r); }
+VARK_DEV void tmem_st_chunk(uint32_t taddr, const uint32_t (&r)[64]) {
+  tmem_st32(taddr, reinterpret_cast<const uint32_t(&)[32]>(r[0]));
+  tmem_st32(taddr + 32, reinterpret_cast<const uint32_t(&)[32]>(r[32]));
+}
 
 template <int D>
 struct Smem {
@@ -280,6 +301,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kc,
             const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ Params p) {
   using L = Smem<D>;
+  using PC = PChunks<MASS, WITH_O>;
   constexpr int QP = L::kQPanels;
   constexpr uint32_t kTileBytes = L::kTile;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -310,7 +332,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(bar(kBarSFull + x), 1);
-      for (int c = 0; c < kPChunks; ++c) mbar_init(bar(kBarPFull + x * kPChunks + c), kBlockM / 32);  // one arrival per warp
+      for (int c = 0; c < kPChunks; ++c) mbar_init(bar(kBarPFull + x * kPChunks + c), PC::kArrivals);
       mbar_init(bar(kBarODone + x), 1);
     }
     mbar_init(bar(kBarDrain), 1);
@@ -363,16 +385,9 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       // ---------------------------------------------------------- producer
       // (Q and the first kStages key tiles were issued right after the
       // barrier initialisation, by this same thread.)
-      // last tile this thread loaded into each stage (-1: none); only those
-      // loads can still be in flight when the loop ends
-      const int first = min(min(n, kStages), p.withhold_tile < 0 ? n : p.withhold_tile);
-      int last_k[kStages], last_v[kStages];
-      for (int st = 0; st < kStages; ++st) {
-        const bool mine = st < first;
-        last_k[st] = mine ? st : -1;
-        last_v[st] = (mine && WITH_O) ? st : -1;
-      }
-      for (int j = first; j < n; ++j) {
+      int issued_k = min(min(n, kStages), p.withhold_tile < 0 ? n : p.withhold_tile);
+      int issued_v = WITH_O ? issued_k : 0;
+      for (int j = issued_k; j < n; ++j) {
         const int st = j % kStages;
         const KTile t = it.tile(p, j);
         if (j == p.withhold_tile) break;   // test hook: this tile never arrives
@@ -383,7 +398,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           if (t.src == 0) tma_load_3d(dst, &tm_k, bar(kBarKFull + st), c * 64, t.row, it.bh);
           else tma_load_2d(dst, &tm_kc, bar(kBarKFull + st), c * 64, t.row);
         }
-        last_k[st] = j;
+        issued_k = j + 1;
         if (!WITH_O) continue;
         if (j >= kStages && !mbar_wait(bar(kBarVEmpty + st), ((j / kStages) - 1) & 1, abort_flag, p.status, p.wait_limit_ns)) break;
         mbar_arrive_expect_tx(bar(kBarVFull + st), kTileBytes);
@@ -392,16 +407,16 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           if (t.src == 0) tma_load_3d(dst, &tm_v, bar(kBarVFull + st), c * 64, t.row, it.bh);
           else tma_load_2d(dst, &tm_vc, bar(kBarVFull + st), c * 64, t.row);
         }
-        last_v[st] = j;
+        issued_v = j + 1;
       }
       // Drain: every load issued here has landed before the CTA exits
       // (immediate on the normal path; bounded on the abort path).
       volatile int no_abort = 0;
       mbar_wait(bar(kBarQ), 0, &no_abort, nullptr);
-      for (int st = 0; st < kStages; ++st) {
-        if (last_k[st] >= 0) mbar_wait(bar(kBarKFull + st), (last_k[st] / kStages) & 1, &no_abort, nullptr);
-        if (last_v[st] >= 0) mbar_wait(bar(kBarVFull + st), (last_v[st] / kStages) & 1, &no_abort, nullptr);
-      }
+      for (int j = max(0, issued_k - kStages); j < issued_k; ++j)
+        mbar_wait(bar(kBarKFull + j % kStages), (j / kStages) & 1, &no_abort, nullptr);
+      for (int j = max(0, issued_v - kStages); j < issued_v; ++j)
+        mbar_wait(bar(kBarVFull + j % kStages), (j / kStages) & 1, &no_abort, nullptr);
     } else if (warp == 1 && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
       constexpr uint32_t idesc_s = idesc_bf16_f32(kBlockM, kBlockN, false, false);
@@ -420,13 +435,13 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       // that chunk.  Returns false on abort.
       auto issue_pv = [&](int x, int pst, int jp) -> bool {
 #pragma unroll
-        for (int c = 0; c < kPChunks; ++c) {
+        for (int c = 0; c < PC::kCount; ++c) {
           if (!mbar_wait(bar(kBarPFull + x * kPChunks + c), jp & 1, abort_flag, p.status, p.wait_limit_ns))
             return false;
           tc_fence_after();
 #pragma unroll
-          for (int kq = 0; kq < kChunkKeys / 16; ++kq) {
-            const int kk = c * (kChunkKeys / 16) + kq;
+          for (int kq = 0; kq < PC::kKeys / 16; ++kq) {
+            const int kk = c * (PC::kKeys / 16) + kq;
             const uint64_t b = smem_desc_sw128(sV + pst * kTileBytes + kk * 2048, kPanelBytes, 1024);
             mma_bf16_ts(tmem + 256 + x * D, tmem + x * kBlockN + kk * 8, b, idesc_o, (jp > 0 || kk > 0) ? 1u : 0u);
           }
@@ -535,8 +550,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       }
       if (!WITH_O) {   // S_X is in registers: the next S MMA of this tile may overwrite it
         tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(kBarPFull + x * kPChunks));
+        mbar_arrive(bar(kBarPFull + x * kPChunks));
       }
       float m_tile, sh;
       if (fast) {
@@ -603,19 +617,19 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           tmem_st32(tO + c * 32, v);
         }
       }
-      // p = 2^(exponent - m_used), one chunk of kChunkKeys columns at a time.
+      // p = 2^(exponent - m_used), one chunk of PC::kKeys columns at a time.
       // With O, chunk q's bf16 pairs go to TMEM (over S_X's first columns)
       // while chunk q+1's exponentials run, and the warp signals the chunk
       // to the MMA thread once its store has completed.
       const float shm = fast ? sh - m_used : -m_used;
 #pragma unroll
-      for (int q = 0; q < kPChunks; ++q) {
-        float* cv = sv + q * kChunkKeys;
+      for (int q = 0; q < PC::kCount; ++q) {
+        float* cv = sv + q * PC::kKeys;
         if (fast) {
 #pragma unroll
-          for (int c = 0; c < kChunkKeys; c += 2) ffma2(cv[c], cv[c + 1], cv[c], cv[c + 1], qk2, qk2, shm, shm);
+          for (int c = 0; c < PC::kKeys; c += 2) ffma2(cv[c], cv[c + 1], cv[c], cv[c + 1], qk2, qk2, shm, shm);
 #pragma unroll
-          for (int c = 0; c < kChunkKeys; c += 8) {
+          for (int c = 0; c < PC::kKeys; c += 8) {
             constexpr int kPoly = WITH_O ? kPolyPer8 : kPolyPer8NoO;
 #pragma unroll
             for (int i = 0; i < kPoly; i += 2) exp2_poly2(cv[c + i], cv[c + i + 1]);
@@ -624,9 +638,9 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           }
         } else {
 #pragma unroll
-          for (int c = 0; c < kChunkKeys; c += 2) fadd2(cv[c], cv[c + 1], cv[c], cv[c + 1], shm, shm);
+          for (int c = 0; c < PC::kKeys; c += 2) fadd2(cv[c], cv[c + 1], cv[c], cv[c + 1], shm, shm);
 #pragma unroll
-          for (int c = 0; c < kChunkKeys; ++c) cv[c] = ex2_approx(cv[c]);
+          for (int c = 0; c < PC::kKeys; ++c) cv[c] = ex2_approx(cv[c]);
         }
         if (WITH_O) {
           if (q > 0) {   // chunk q-1's store has been in flight during these exponentials
@@ -635,17 +649,21 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(kBarPFull + x * kPChunks + q - 1));
           }
-          uint32_t pk[kChunkKeys / 2];
+          uint32_t pk[PC::kKeys / 2];
 #pragma unroll
-          for (int c = 0; c < kChunkKeys / 2; ++c) pk[c] = pack_bf16x2(cv[2 * c], cv[2 * c + 1]);
-          tmem_st16(tS + q * (kChunkKeys / 2), pk);
+          for (int c = 0; c < PC::kKeys / 2; ++c) pk[c] = pack_bf16x2(cv[2 * c], cv[2 * c + 1]);
+          tmem_st_chunk(tS + q * (PC::kKeys / 2), pk);
         }
       }
       if (WITH_O) {
         tmem_wait_st();
         tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(kBarPFull + x * kPChunks + kPChunks - 1));
+        if (PC::kPerWarp) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(kBarPFull + x * kPChunks + PC::kCount - 1));
+        } else {
+          mbar_arrive(bar(kBarPFull + x * kPChunks + PC::kCount - 1));
+        }
       }
       float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f, a4 = 0.f, a5 = 0.f, a6 = 0.f, a7 = 0.f;
 #pragma unroll

@@ -371,8 +371,6 @@ constexpr int kQuantCluster = 8;
 constexpr int kQuantGroupLH = 2048;  // (layer, head) pairs per launch group
 constexpr int kSmallRows = 1024;
 constexpr int kQuantMaxD = 512;
-// 0: single-read cluster kernel; 1: two streaming passes (absmax, then codes).
-constexpr bool kQuantTwoPass = false;
 
 struct QuantParams {
   ScaleTable sc;
@@ -684,207 +682,6 @@ __global__ void __cluster_dims__(kQuantCluster, 1, 1) __launch_bounds__(kQuantTh
   cluster_sync_all();   // no CTA leaves while a peer may still read its partial maxima
 }
 
-// Two-pass quantisation.  Pass 1 (absmax_kernel): one CTA per (block,
-// tensor), big blocks first, streams the block once and writes its table
-// entries in their final form (fp32 absmax, or the bf16 scale of 4-bit codes)
-// -- no cross-CTA reduction, no atomics.  Pass 2 (codes_kernel): a pure stream
-// over (block, 64-row chunk) units in memory order, like the compaction; each
-// unit reads its 8 channels' table entries (L2-resident) and writes codes.
-// The kept bf16 bytes are read twice from HBM, but neither pass ever waits on
-// another CTA.
-constexpr int kAbsThreads = 256;
-constexpr int kCodeRows = 64;
-constexpr int kCodeThreads = 256;
-
-template <int BITS>
-__global__ void __launch_bounds__(kAbsThreads, 4) absmax_kernel(
-    const uint4* __restrict__ k, const uint4* __restrict__ v, QuantParams p, const uint8_t* __restrict__ keep,
-    void* __restrict__ ka, void* __restrict__ va) {
-  __shared__ int32_t big_prefix[kQuantGroupLH + 1];
-  __shared__ int32_t small_prefix[kQuantGroupLH + 1];
-  __shared__ uint32_t keep_mask[kQuantGroupLH];
-  __shared__ int32_t warp_tot[kAbsThreads / 32];
-  __shared__ __align__(16) uint32_t red[kAbsThreads * 4];
-  const int S = p.sc.S, H = p.H, D = p.D, B = p.B;
-  const int nlh = p.nl * H;
-  const int lh0 = p.l0 * H;
-  for (int i = threadIdx.x; i < nlh; i += kAbsThreads) {
-    const uint8_t* kp = keep + int64_t(lh0 + i) * S;
-    uint32_t m = 0;
-    for (int s = 0; s < S; ++s)
-      if (kp[s]) m |= 1u << s;
-    keep_mask[i] = m;
-    big_prefix[i] = __popc(m & p.big_mask);
-    small_prefix[i] = __popc(m & ~p.big_mask);
-  }
-  __syncthreads();
-  block_exclusive_scan<kAbsThreads, kQuantGroupLH>(big_prefix, nlh, warp_tot);
-  block_exclusive_scan<kAbsThreads, kQuantGroupLH>(small_prefix, nlh, warp_tot);
-  const int64_t n_big = int64_t(big_prefix[nlh]) * 2 * B;
-  const int64_t n_units = n_big + int64_t(small_prefix[nlh]) * 2 * B;
-  const int cv_n = D / 8;
-  const int nrg = kAbsThreads / cv_n;
-  const bool active = threadIdx.x < nrg * cv_n;
-  const int cv = threadIdx.x % cv_n;
-  const int rg = threadIdx.x / cv_n;
-  for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x) {
-    const bool big = u < n_big;
-    const QBlock q = big ? decode_block(u, big_prefix, keep_mask, p.big_mask, p)
-                         : decode_block(u - n_big, small_prefix, keep_mask, ~p.big_mask, p);
-    const int32_t nr = p.sc.n[q.s];
-    const uint4* src = (q.t ? v : k) +
-                       (int64_t(q.l) * p.layer_stride + ((int64_t(q.b) * H + q.h) * p.sc.T + p.sc.off[q.s]) * D) / 8 +
-                       cv;
-    uint32_t acc[4] = {0u, 0u, 0u, 0u};
-    if (active) {
-      int32_t r = rg;
-      for (; r + 7 * nrg < nr; r += 8 * nrg) {
-        uint4 x[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = __ldcs(src + int64_t(r + e * nrg) * cv_n);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) absmax8(acc, x[e]);
-      }
-      for (; r < nr; r += nrg) absmax8(acc, __ldcs(src + int64_t(r) * cv_n));
-      *reinterpret_cast<uint4*>(&red[threadIdx.x * 4]) = make_uint4(acc[0], acc[1], acc[2], acc[3]);
-    }
-    __syncthreads();
-    const int dw = D / 2;
-    const int64_t t0 = ((((int64_t(q.l) * B + q.b) * H + q.h) * S) + q.s) * D;
-    for (int x = threadIdx.x; x < dw; x += kAbsThreads) {   // channel pair x: entries red[e * dw + x]
-      uint32_t w = 0;
-      for (int e = 0; e < nrg; ++e) w = __vmaxu2(w, red[e * dw + x]);
-      const float a0 = lo_bf16(w), a1 = hi_bf16(w);
-      if (BITS == 8) {
-        float* t = static_cast<float*>(q.t ? va : ka) + t0;
-        t[2 * x] = a0;
-        t[2 * x + 1] = a1;
-      } else {
-        const uint32_t s0 = __float_as_uint(make_qscale<4>(a0).sc) >> 16, s1 = __float_as_uint(make_qscale<4>(a1).sc) >> 16;
-        reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(q.t ? va : ka) + t0)[x] = s0 | (s1 << 16);
-      }
-    }
-    __syncthreads();   // red is rewritten by the next unit
-  }
-}
-
-template <int BITS>
-__global__ void __launch_bounds__(kCodeThreads, 4) codes_kernel(
-    const uint4* __restrict__ k, const uint4* __restrict__ v, CompactParams p, const uint8_t* __restrict__ keep,
-    const int32_t* __restrict__ head_off, const int32_t* __restrict__ seg_off, const int64_t* __restrict__ layer_base,
-    void* __restrict__ kq, void* __restrict__ vq, const void* __restrict__ ka, const void* __restrict__ va) {
-  __shared__ int32_t chunk_prefix[kMaxGroupLH + 1];
-  __shared__ uint32_t keep_mask[kMaxGroupLH];
-  __shared__ int32_t warp_tot[kCodeThreads / 32];
-  const int S = p.sc.S, H = p.H, D = p.D, B = p.B;
-  const int nlh = p.nl * H;
-  const int lh0 = p.l0 * H;
-  for (int i = threadIdx.x; i < nlh; i += kCodeThreads) {
-    const uint8_t* kp = keep + int64_t(lh0 + i) * S;
-    uint32_t m = 0;
-    int32_t c = 0;
-    for (int s = 0; s < S; ++s)
-      if (kp[s]) {
-        m |= 1u << s;
-        c += (p.sc.n[s] + kCodeRows - 1) / kCodeRows;
-      }
-    keep_mask[i] = m;
-    chunk_prefix[i] = c;
-  }
-  __syncthreads();
-  block_exclusive_scan<kCodeThreads, kMaxGroupLH>(chunk_prefix, nlh, warp_tot);
-  const int32_t grand = chunk_prefix[nlh];
-  const int64_t units = int64_t(grand) * B * 2;     // (layer, batch, head, chunk) x {K, V}
-  const int cv_n = D / 8;
-  const int nrg = kCodeThreads / cv_n;
-  if (threadIdx.x >= nrg * cv_n) return;            // no block-wide barrier follows
-  const int cv = threadIdx.x % cv_n;
-  const int rg = threadIdx.x / cv_n;
-  for (int64_t g2 = blockIdx.x; g2 < units; g2 += gridDim.x) {
-    const int t = int(g2 & 1);
-    const int64_t g = g2 >> 1;
-    int la = 0, lz = p.nl;
-    while (lz - la > 1) {
-      const int mid = (la + lz) >> 1;
-      if (int64_t(chunk_prefix[mid * H]) * B <= g) la = mid; else lz = mid;
-    }
-    const int32_t c0 = chunk_prefix[la * H];
-    const int32_t C = chunk_prefix[(la + 1) * H] - c0;
-    const int64_t r = g - int64_t(c0) * B;
-    const int b = int(r / C);
-    const int32_t c = c0 + int32_t(r % C);
-    int lo = la * H, hi = (la + 1) * H;
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (chunk_prefix[mid] <= c) lo = mid; else hi = mid;
-    }
-    int32_t j = c - chunk_prefix[lo];
-    const uint32_t m = keep_mask[lo];
-    int s = 0;
-    for (; s < S; ++s)
-      if (m >> s & 1u) {
-        const int32_t ch = (p.sc.n[s] + kCodeRows - 1) / kCodeRows;
-        if (j < ch) break;
-        j -= ch;
-      }
-    const int l = p.l0 + lo / H;
-    const int h = lo % H;
-    const int32_t r0 = j * kCodeRows;
-    const int32_t nrows = min(kCodeRows, p.sc.n[s] - r0);
-    // the 8 channels' scales of this block
-    const int64_t t0 = ((((int64_t(l) * B + b) * H + h) * S) + s) * D + cv * 8;
-    float sc[8], rc[8];
-    if (BITS == 8) {
-      const float* tab = static_cast<const float*>(t ? va : ka) + t0;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const QScale qs = make_qscale<8>(tab[e]);
-        sc[e] = qs.sc;
-        rc[e] = qs.rc;
-      }
-    } else {
-      const uint4 w = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(t ? va : ka) + t0);
-      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        sc[2 * e] = lo_bf16(ww[e]);
-        sc[2 * e + 1] = hi_bf16(ww[e]);
-      }
-#pragma unroll
-      for (int e = 0; e < 8; ++e) rc[e] = (sc[e] >= 0x1p-100f && sc[e] <= 0x1p100f) ? __frcp_rn(sc[e]) : 0.f;
-    }
-    bool force = false;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) force |= sc[e] != 0.f && rc[e] == 0.f;
-    const uint4* src = (t ? v : k) +
-                       (int64_t(l) * p.layer_stride + ((int64_t(b) * H + h) * p.sc.T + p.sc.off[s] + r0) * D) / 8 + cv;
-    const int64_t R_l = (layer_base[l + 1] - layer_base[l]) / (int64_t(B) * D);
-    const int64_t e_first = layer_base[l] + (int64_t(b) * R_l + head_off[l * H + h] + seg_off[(l * H + h) * S + s] + r0) * D;
-    int32_t rr = rg;
-    if (BITS == 8) {
-      uint2* dst = reinterpret_cast<uint2*>(static_cast<int8_t*>(t ? vq : kq) + e_first) + cv;
-      for (; rr + 3 * nrg < nrows; rr += 4 * nrg) {
-        uint4 x[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) x[e] = __ldcs(src + (rr + e * nrg) * cv_n);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) __stcs(dst + (rr + e * nrg) * cv_n, codes8(x[e], sc, rc, force));
-      }
-      for (; rr < nrows; rr += nrg) __stcs(dst + rr * cv_n, codes8(__ldcs(src + rr * cv_n), sc, rc, force));
-    } else {
-      uint32_t* dst = static_cast<uint32_t*>(t ? vq : kq) + e_first / 8 + cv;
-      for (; rr + 3 * nrg < nrows; rr += 4 * nrg) {
-        uint4 x[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) x[e] = __ldcs(src + (rr + e * nrg) * cv_n);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) __stcs(dst + (rr + e * nrg) * cv_n, codes4x8(x[e], sc, rc, force));
-      }
-      for (; rr < nrows; rr += nrg) __stcs(dst + rr * cv_n, codes4x8(__ldcs(src + rr * cv_n), sc, rc, force));
-    }
-  }
-}
-
 // Dequantisation of one layer.  Unit = (batch, head, kept scale, chunk of at
 // most kDeqRows rows), in that (memory) order; each thread keeps the scales of
 // its 8 channels for the unit and streams rows, four at a time: 8-byte code
@@ -1087,24 +884,6 @@ static int quantize_kv(const uint16_t* k, const uint16_t* v, int64_t layer_strid
     clusters = std::max(1, nsm / kQuantCluster);
   }
   const int layers_per_group = std::max(1, kQuantGroupLH / H);
-  if (kQuantTwoPass) {
-    CompactParams cp;
-    cp.sc = q.sc;
-    cp.L = L; cp.B = B; cp.H = H; cp.D = D; cp.layer_stride = layer_stride;
-    const int groups2 = std::max(1, std::min(layers_per_group, kMaxGroupLH / H));
-    for (int l0 = 0; l0 < L; l0 += groups2) {
-      q.l0 = cp.l0 = l0;
-      q.nl = cp.nl = std::min(groups2, L - l0);
-      absmax_kernel<BITS><<<nsm * 4, kAbsThreads, 0, st>>>(reinterpret_cast<const uint4*>(k),
-                                                           reinterpret_cast<const uint4*>(v), q, keep, k_tab, v_tab);
-      if (cudaGetLastError() != cudaSuccess) return VARK_E_CUDA;
-      codes_kernel<BITS><<<nsm * 4, kCodeThreads, 0, st>>>(
-          reinterpret_cast<const uint4*>(k), reinterpret_cast<const uint4*>(v), cp, keep, head_off, seg_off,
-          layer_base, kq, vq, k_tab, v_tab);
-      if (cudaGetLastError() != cudaSuccess) return VARK_E_CUDA;
-    }
-    return VARK_OK;
-  }
   for (int l0 = 0; l0 < L; l0 += layers_per_group) {
     q.l0 = l0;
     q.nl = std::min(layers_per_group, L - l0);
