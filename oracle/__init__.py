@@ -36,7 +36,8 @@ from .generation import append_scale, cache_size_after_layer
 from .stability import rank_stability, average_ranks
 from .early_pruning import early_pruning_schedule, keep_after_step
 from .quant import (quantize_block, dequantize_block, quantize_kv, quantize_block_int4, dequantize_block_int4,
-                    pack_int4, unpack_int4, quantize_kv_int4, int4_scale_bits)
+                    pack_int4, unpack_int4, quantize_kv_int4, int4_scale_bits, quantize_block_int3,
+                    dequantize_block_int3, pack_int3, unpack_int3, quantize_kv_int3, int3_scale_bits)
 
 __all__ = [
     "ScaleGeometry", "block_causal_attention", "attend", "scas_mass", "pruned_attention",
@@ -44,5 +45,6 @@ __all__ = [
     "build_offsets", "compact_kv", "append_scale", "cache_size_after_layer",
     "rank_stability", "average_ranks", "early_pruning_schedule", "keep_after_step",
     "quantize_block", "dequantize_block", "quantize_kv", "quantize_block_int4", "dequantize_block_int4",
-    "pack_int4", "unpack_int4", "quantize_kv_int4", "int4_scale_bits",
+    "pack_int4", "unpack_int4", "quantize_kv_int4", "int4_scale_bits", "quantize_block_int3",
+    "dequantize_block_int3", "pack_int3", "unpack_int3", "quantize_kv_int3", "int3_scale_bits",
 ]

@@ -821,3 +821,108 @@ def test_quantize_kv_int4_identity_coded():
                         want = want_codes[l, b, h, g.off[s] + t]
                         assert np.array_equal(got_k, want) and np.array_equal(got_v, -want), (l, b, h, s, t)
         base += B * int(R[l].sum()) * D
+
+
+# ---------------------------------------------------------------- 3-bit retained cache
+
+def test_int3_block_quantisation_pins():
+    from synth import f32_to_bf16_bits
+    rng = np.random.default_rng(46)
+    x = f32_to_bf16_bits(rng.standard_normal((300, 16)).astype(np.float32) * 3)
+    codes, s_bits = oracle.quantize_block_int3(x)
+    s = bf16_bits_to_f32(s_bits).astype(np.float64)
+    a = np.abs(bf16_bits_to_f32(x)).max(axis=0).astype(np.float64)
+    # s is a / 3 rounded to bf16: within half a bf16 step of it
+    assert np.all(np.abs(s - a / 3.0) <= (a / 3.0) * 2.0 ** -8)
+    back = bf16_bits_to_f32(oracle.dequantize_block_int3(codes, s_bits)).astype(np.float64)
+    xf = bf16_bits_to_f32(x).astype(np.float64)
+    assert np.all(np.abs(back - xf) <= s[None, :] / 2.0 + np.abs(back) * 2.0 ** -9 + 1e-12)
+    assert np.all(np.abs(codes.astype(np.int64)).max(axis=0) == 3)       # the absmax element maps to +-3
+    assert codes.min() >= -3 and codes.max() <= 3
+    # the exact product, rounded once: code * s has at most 10 significant bits
+    prod = codes.astype(np.float64) * s[None, :]
+    assert np.array_equal(oracle.dequantize_block_int3(codes, s_bits),
+                          f32_to_bf16_bits(prod.astype(np.float32)))
+    # integers in [-3, 3] with absmax 3 on every channel: scale 1, exact round trip
+    ints = rng.integers(-3, 4, size=(40, 8)).astype(np.float32)
+    ints[0] = -3.0
+    xi = f32_to_bf16_bits(ints)
+    ci, si = oracle.quantize_block_int3(xi)
+    assert np.all(bf16_bits_to_f32(si) == 1.0)
+    assert np.array_equal(ci.astype(np.float32), ints) and np.array_equal(oracle.dequantize_block_int3(ci, si), xi)
+    # halves round to even: with scale 1, 0.5 -> 0, 1.5 -> 2, -2.5 -> -2
+    xh = f32_to_bf16_bits(np.array([[0.5, 1.5, -2.5, 3.0], [3.0, -3.0, 3.0, -3.0]], dtype=np.float32))
+    ch, sh = oracle.quantize_block_int3(xh)
+    assert np.all(bf16_bits_to_f32(sh) == 1.0) and ch[0].tolist() == [0, 2, -2, 3]
+    # zero block
+    cz, sz = oracle.quantize_block_int3(np.zeros((4, 8), dtype=np.uint16))
+    assert not cz.any() and not sz.any() and not oracle.dequantize_block_int3(cz, sz).any()
+
+
+def test_int3_packing_layout():
+    """One hand-packed group: codes c0..c7 = -3, -2, -1, 0, 1, 2, 3, 0 give
+    fields 1, 2, 3, 4, 5, 6, 7, 4 at bits 3j; written high field first that is
+    100 111 110 101 100 011 010 001 = 0x9F58D1, stored little-endian.  A second
+    group follows in the next three bytes."""
+    codes = np.array([[-3, -2, -1, 0, 1, 2, 3, 0, 3, 3, 3, 3, 3, 3, 3, 3]], dtype=np.int8)
+    packed = oracle.pack_int3(codes)
+    assert packed.tolist() == [[0xD1, 0x58, 0x9F, 0xFF, 0xFF, 0xFF]]   # eight 7-fields = 24 ones
+    rng = np.random.default_rng(47)
+    many = rng.integers(-3, 4, size=(33, 64)).astype(np.int8)
+    assert np.array_equal(oracle.unpack_int3(oracle.pack_int3(many), 64), many)
+
+
+def test_quantize_kv_int3_identity_coded():
+    """Integer codes in [-3, 3] times a power-of-two unit per block, one +-3
+    element per channel: the codes are the integers, the scale the unit, and
+    every 3-bit field must land at its compacted position (byte 3 e / 8)."""
+    from synth import f32_to_bf16_bits
+    sides = SIDES_TINY
+    g = _geom(sides)
+    L, B, H, D = 2, 2, 3, 16
+    T = g.T
+    keep = np.random.default_rng(14).integers(0, 2, size=(L, H, g.S)).astype(np.uint8)
+    keep[1, 2, :] = 1
+
+    def code(l, b, h, t, d):
+        return int((l * 5 + b * 11 + h * 3 + t * 7 + d * 13) % 7) - 3
+
+    def unit(l, b, h, s):
+        return 2.0 ** (((3 * l + b + 2 * h + s) % 9) - 4)
+
+    dense = np.zeros((L, B, H, T, D), dtype=np.float32)
+    want_codes = np.zeros((L, B, H, T, D), dtype=np.int64)
+    for l in range(L):
+        for b in range(B):
+            for h in range(H):
+                for s in range(g.S):
+                    for t in range(g.off[s], g.off[s] + g.n[s]):
+                        for d in range(D):
+                            c = code(l, b, h, t, d)
+                            if (t - g.off[s]) == d % g.n[s]:
+                                c = 3 if (d + t) % 2 == 0 else -3
+                            want_codes[l, b, h, t, d] = c
+                            dense[l, b, h, t, d] = c * unit(l, b, h, s)
+    kb = f32_to_bf16_bits(dense)
+    vb = f32_to_bf16_bits(-dense)
+    head_off, seg_off, _, layer_base = oracle.build_offsets(keep, sides, B, D)
+    kq, vq, ks, vs = oracle.quantize_kv_int3(kb, vb, keep, sides, head_off, seg_off, layer_base)
+    R = (keep * np.array(g.n)[None, None, :]).sum(axis=2)
+    assert 8 * kq.size == 3 * sum(B * int(R[l].sum()) * D for l in range(L))
+    base = 0
+    for l in range(L):
+        for b in range(B):
+            for h in range(H):
+                for s in range(g.S):
+                    if not keep[l, h, s]:
+                        assert not ks[l, b, h, s].any() and not vs[l, b, h, s].any()
+                        continue
+                    assert np.all(bf16_bits_to_f32(ks[l, b, h, s]) == unit(l, b, h, s))
+                    row0 = b * int(R[l].sum()) + int(R[l, :h].sum()) + sum(g.n[t] for t in range(s) if keep[l, h, t])
+                    for t in range(g.n[s]):
+                        lo = 3 * (base + (row0 + t) * D) // 8
+                        got_k = oracle.unpack_int3(kq[lo:lo + 3 * D // 8], D)[0]
+                        got_v = oracle.unpack_int3(vq[lo:lo + 3 * D // 8], D)[0]
+                        want = want_codes[l, b, h, g.off[s] + t]
+                        assert np.array_equal(got_k, want) and np.array_equal(got_v, -want), (l, b, h, s, t)
+        base += B * int(R[l].sum()) * D
