@@ -555,18 +555,21 @@ def int8_cache(pipe, max_over_ranks, bf16_attention_ms, hbm_gbs, reps=3):
             "bf16_cache_attention_ms": bf16_attention_ms}
 
 
-def int4_cache(pipe, max_over_ranks, bf16_attention_ms, hbm_gbs, reps=3):
-    """The retained cache stored as packed 4-bit codes with per-(block,
-    channel) bf16 scales: quantising compaction of all layers, then per layer
-    dequantisation into a one-layer bf16 buffer followed by that layer's
-    pruned attention."""
+def packed_cache(pipe, max_over_ranks, bf16_attention_ms, hbm_gbs, bits, reps=3):
+    """The retained cache stored as packed 4-bit or 3-bit codes with
+    per-(block, channel) bf16 scales: quantising compaction of all layers,
+    then per layer dequantisation into a one-layer bf16 buffer followed by
+    that layer's pruned attention."""
     import torch
     vark, w = pipe.vark, pipe.w
     L, B, H, D, S, T = w.layers, w.batch, w.heads, w.head_dim, pipe.S, pipe.T
+    num, den = {4: (1, 2), 3: (3, 8)}[bits]      # code bytes per element
+    quantize = {4: vark.vark_quantize_kv_int4, 3: vark.vark_quantize_kv_int3}[bits]
+    dequantize = {4: vark.vark_dequantize_layer_int4, 3: vark.vark_dequantize_layer_int3}[bits]
     base = pipe.base_host.numpy()
     total = int(base[-1])
     dev = pipe.dev
-    kq = torch.empty(max(total // 2, 16), dtype=torch.uint8, device=dev)
+    kq = torch.empty(max(num * total // den, 16), dtype=torch.uint8, device=dev)
     vq = torch.empty_like(kq)
     ks = torch.empty((L, B, H, S, D), dtype=torch.int16, device=dev)
     vs = torch.empty_like(ks)
@@ -578,23 +581,23 @@ def int4_cache(pipe, max_over_ranks, bf16_attention_ms, hbm_gbs, reps=3):
 
     def one():
         ev[0].record(st)
-        vark.vark_quantize_kv_int4(pipe.k, pipe.v, B * H * T * D, L, B, H, pipe.sides, D, pipe.keep, pipe.head_off,
-                                   pipe.seg_off, pipe.layer_base, kq, vq, ks, vs)
+        quantize(pipe.k, pipe.v, B * H * T * D, L, B, H, pipe.sides, D, pipe.keep, pipe.head_off, pipe.seg_off,
+                 pipe.layer_base, kq, vq, ks, vs)
         ev[1].record(st)
         for l in range(L):
             rows = int(base[l + 1] - base[l]) // D
-            b0 = int(base[l]) // 2
-            vark.vark_dequantize_layer_int4(kq[b0:], vq[b0:], ks[l], vs[l], rows, B, H, pipe.sides, D,
-                                            pipe.head_off[l], pipe.seg_off[l], kcl, vcl)
+            b0 = num * int(base[l]) // den
+            dequantize(kq[b0:], vq[b0:], ks[l], vs[l], rows, B, H, pipe.sides, D, pipe.head_off[l],
+                       pipe.seg_off[l], kcl, vcl)
             vark.vark_pruned_attention(pipe.q[l], kcl if rows else None, vcl if rows else None, rows, pipe.k[l],
                                        pipe.v[l], pipe.sides, -1, pipe.head_off[l], pipe.seg_off[l],
                                        pipe.past_len[l], pipe.tau[l], pipe.bias[l], pipe.out[l], pipe.status)
         ev[2].record(st)
         for l in range(L):     # the dequantisations alone
             rows = int(base[l + 1] - base[l]) // D
-            b0 = int(base[l]) // 2
-            vark.vark_dequantize_layer_int4(kq[b0:], vq[b0:], ks[l], vs[l], rows, B, H, pipe.sides, D,
-                                            pipe.head_off[l], pipe.seg_off[l], kcl, vcl)
+            b0 = num * int(base[l]) // den
+            dequantize(kq[b0:], vq[b0:], ks[l], vs[l], rows, B, H, pipe.sides, D, pipe.head_off[l],
+                       pipe.seg_off[l], kcl, vcl)
         ev[3].record(st)
 
     one()
@@ -609,9 +612,10 @@ def int4_cache(pipe, max_over_ranks, bf16_attention_ms, hbm_gbs, reps=3):
     assert int(pipe.status.item()) == 0
     tq, ta, td = max_over_ranks(tq / reps), max_over_ranks(ta / reps), max_over_ranks(td / reps)
     bf16_bytes = 2 * 2 * total
-    int4_bytes = 2 * (total // 2) + 2 * 2 * ks.numel()
-    q_bytes = bf16_bytes + int4_bytes     # kept bf16 K, V read once; packed codes and scale tables written
-    return {"cache_bytes_bf16": bf16_bytes, "cache_bytes_int4": int4_bytes, "cache_ratio": int4_bytes / bf16_bytes,
+    packed_bytes = 2 * (num * total // den) + 2 * 2 * ks.numel()
+    q_bytes = bf16_bytes + packed_bytes   # kept bf16 K, V read once; packed codes and scale tables written
+    return {"cache_bytes_bf16": bf16_bytes, f"cache_bytes_int{bits}": packed_bytes,
+            "cache_ratio": packed_bytes / bf16_bytes,
             "quantize_ms": tq * 1e3, "quantize_gbs": q_bytes / tq / 1e9,
             "quantize_frac_of_hbm": q_bytes / tq / 1e9 / hbm_gbs,
             "dequantize_ms": td * 1e3, "dequantize_gbs": q_bytes / td / 1e9,
@@ -962,7 +966,7 @@ def early_pruning_order(pipe, per_scale, outs, passes, max_over_ranks, sum_over_
             "bytes_moved_per_pass": moved}
 
 
-def summarize_kernels(kernels, quant, quant4, others, scas_o, peaks):
+def summarize_kernels(kernels, quant, quant4, quant3, others, scas_o, peaks):
     """Rounded per-kernel rates and roofline fractions (sustained / burst)."""
     bs, bb, hb = peaks["bf16_tflops_sustained"], peaks["bf16_tflops"], peaks["hbm_gbs"]
     r = lambda x: None if x is None else round(float(x), 3)
@@ -983,6 +987,10 @@ def summarize_kernels(kernels, quant, quant4, others, scas_o, peaks):
         out["int4"] = {"cache_ratio": r(quant4["cache_ratio"]), "quantize_frac_of_hbm": r(quant4["quantize_frac_of_hbm"]),
                        "dequantize_frac_of_hbm": r(quant4["dequantize_frac_of_hbm"]),
                        "dequant_plus_attention_vs_bf16": r(quant4["dequant_plus_attention_ms"] / quant4["bf16_cache_attention_ms"])}
+    if quant3:
+        out["int3"] = {"cache_ratio": r(quant3["cache_ratio"]), "quantize_frac_of_hbm": r(quant3["quantize_frac_of_hbm"]),
+                       "dequantize_frac_of_hbm": r(quant3["dequantize_frac_of_hbm"]),
+                       "dequant_plus_attention_vs_bf16": r(quant3["dequant_plus_attention_ms"] / quant3["bf16_cache_attention_ms"])}
     if others:
         l8 = others["large_8l"]
         out["large_8l"] = {"calibration_tflops": r(l8["calibration_tflops"]), "pruned_tflops": r(l8["pruned_attention_tflops"]),
@@ -1254,7 +1262,8 @@ def main():
 
     # ------------------------------------------------ int8 retained cache
     quant = int8_cache(pipe, max_over_ranks, ph["attn"] * 1e3 / K, peaks["hbm_gbs"]) if args.quant else None
-    quant4 = int4_cache(pipe, max_over_ranks, ph["attn"] * 1e3 / K, peaks["hbm_gbs"]) if args.quant else None
+    quant4 = packed_cache(pipe, max_over_ranks, ph["attn"] * 1e3 / K, peaks["hbm_gbs"], 4) if args.quant else None
+    quant3 = packed_cache(pipe, max_over_ranks, ph["attn"] * 1e3 / K, peaks["hbm_gbs"], 3) if args.quant else None
 
     # ------------------------------------------------ generation order (scale by scale)
     gen = None
@@ -1289,7 +1298,7 @@ def main():
     # travel with the headline fields.  Convention: kernels timed inside the
     # step are set against the sustained bf16 peak, single launches timed
     # alone against the burst peak; both fractions are given for each.
-    roof["per_kernel"] = summarize_kernels(kernels, quant, quant4, others, scas_o, peaks)
+    roof["per_kernel"] = summarize_kernels(kernels, quant, quant4, quant3, others, scas_o, peaks)
 
     if rank == 0:
         line = {
@@ -1299,7 +1308,7 @@ def main():
             "config": arm_config(w, world),
             "pruned_attention_tflops": pruned_tflops, "query_tokens_per_s": qtok_s, "compaction_gbs": comp_gbs,
             "roofline": roof, "kernels": kernels, "generation_order": gen, "ranking_stability": stab,
-            "int8_cache": quant, "int4_cache": quant4, "other_configs": others, "scas_without_output": scas_o,
+            "int8_cache": quant, "int4_cache": quant4, "int3_cache": quant3, "other_configs": others, "scas_without_output": scas_o,
             "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches,
             "clocks": clk, "peaks": peaks,

@@ -428,6 +428,50 @@ int vark_dequantize_layer_int4(const uint8_t* kq, const uint8_t* vq, const uint1
                                const int32_t* sides, const int32_t* head_off, const int32_t* seg_off,
                                uint16_t* kc, uint16_t* vc, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Quantised retained cache (3-bit).  [VAR-Q] summary page, Main Findings: INT3
+ * codes on the (block, channel) groups stay within one FID point of BF16; Key
+ * Contributions: packing realises the saving (up to 78.5% of the KV cache).
+ * Same groups; per channel:
+ *   a    = max |x| over the block        s = bf16(a / 3)   (IEEE fp32 division, RNE to bf16)
+ *   code = rint(x / s) in [-3, 3]        (IEEE fp32 division, half to even; s = 0 gives 0)
+ *   x'   = bf16(code * s)                (the product is exact in fp32; one rounding)
+ * Packing: field = code + 4 (1..7); the 8 channels c0..c7 of a row that start
+ * at a multiple of 8 form one little-endian 24-bit group (3 bytes) with cj in
+ * bits 3j .. 3j + 2.  Element e of the compacted layout (e a multiple of 8)
+ * starts group e / 8 at byte 3 e / 8, so a layer's codes start at byte
+ * 3 layer_base[l] / 8 and a row is 3 D / 8 bytes.  Scale tables are
+ * [L][B][H][S][D] bf16 bits (0 for dropped scales).
+ * ------------------------------------------------------------------------- */
+
+/*
+ * vark_quantize_kv_int3 -- device.  Compaction with 3-bit quantisation: like
+ * vark_quantize_kv_int4, but kq / vq receive 24-bit groups (3 layer_base[L] / 8
+ * bytes each) and k_scale / v_scale the bf16 scales s = bf16(a / 3).  k, v,
+ * kq, vq, k_scale, v_scale 16-byte aligned; layer_stride a multiple of 8.
+ * Errors: VARK_E_ARG, VARK_E_SHAPE (D % 8 != 0, D > 512, H > 2048), VARK_E_ALIGN,
+ * VARK_E_CUDA.
+ */
+int vark_quantize_kv_int3(const uint16_t* k, const uint16_t* v, int64_t layer_stride,
+                          int L, int B, int H, int S, int D, const int32_t* sides,
+                          const uint8_t* keep, const int32_t* head_off, const int32_t* seg_off,
+                          const int64_t* layer_base, uint8_t* kq, uint8_t* vq,
+                          uint16_t* k_scale, uint16_t* v_scale, void* stream);
+
+/*
+ * vark_dequantize_layer_int3 -- device.  Expands one layer's 3-bit codes to
+ * its bf16 compacted block (as vark_dequantize_layer_int8).
+ *   kq, vq        dev uint8, the layer's packed codes (kq + 3 layer_base[l] / 8),
+ *                 kc_rows rows of 3 D / 8 bytes; any alignment.
+ *   k_scale, v_scale  dev bf16 bits [B][H][S][D], the layer's scale tables.
+ *   other arguments as vark_dequantize_layer_int8.
+ * Errors: as vark_dequantize_layer_int8.
+ */
+int vark_dequantize_layer_int3(const uint8_t* kq, const uint8_t* vq, const uint16_t* k_scale,
+                               const uint16_t* v_scale, int64_t kc_rows, int B, int H, int S, int D,
+                               const int32_t* sides, const int32_t* head_off, const int32_t* seg_off,
+                               uint16_t* kc, uint16_t* vc, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -58,6 +58,8 @@ _SIGNATURES = {
     "vark_dequantize_layer_int8": (_I, [_P, _P, _P, _P, _I64, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "vark_quantize_kv_int4": (_I, [_P, _P, _I64, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "vark_dequantize_layer_int4": (_I, [_P, _P, _P, _P, _I64, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
+    "vark_quantize_kv_int3": (_I, [_P, _P, _I64, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "vark_dequantize_layer_int3": (_I, [_P, _P, _P, _P, _I64, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
 }
 
 
@@ -481,3 +483,43 @@ def vark_dequantize_layer_int4(kq, vq, k_scale, v_scale, kc_rows: int, B: int, H
         _dptr(kc, torch.bfloat16, "kc"), _dptr(vc, torch.bfloat16, "vc"), _stream(stream))
     _check(rc, "vark_dequantize_layer_int4")
 
+
+def vark_quantize_kv_int3(k, v, layer_stride: int, L: int, B: int, H: int, sides, D: int, keep, head_off, seg_off,
+                          layer_base, kq, vq, k_scale, v_scale, stream=None):
+    """Device: compaction into 3-bit codes (24-bit groups of 8 channels) +
+    per-(block, channel) bf16 scales (kq / vq must hold 3 layer_base[L] / 8 bytes)."""
+    import torch
+    _layer_tables(keep, head_off, seg_off, layer_base, L, H, sides)
+    _dense_source(k, v, layer_stride, L, B * H * _tokens(sides) * D)
+    _need(k_scale, "k_scale", numel=L * B * H * len(sides) * D)
+    _need(v_scale, "v_scale", numel=L * B * H * len(sides) * D)
+    s_arr, s_ptr = _sides_arg(sides)
+    rc = _load().vark_quantize_kv_int3(
+        _dptr(k, torch.bfloat16, "k"), _dptr(v, torch.bfloat16, "v"), int(layer_stride), int(L), int(B), int(H),
+        len(s_arr), int(D), s_ptr, _dptr(keep, torch.uint8, "keep"), _dptr(head_off, torch.int32, "head_off"),
+        _dptr(seg_off, torch.int32, "seg_off"), _dptr(layer_base, torch.int64, "layer_base"),
+        _dptr(kq, torch.uint8, "kq"), _dptr(vq, torch.uint8, "vq"), _dptr(k_scale, torch.int16, "k_scale"),
+        _dptr(v_scale, torch.int16, "v_scale"), _stream(stream))
+    _check(rc, "vark_quantize_kv_int3")
+
+
+def vark_dequantize_layer_int3(kq, vq, k_scale, v_scale, kc_rows: int, B: int, H: int, sides, D: int, head_off,
+                               seg_off, kc, vc, stream=None):
+    """Device: one layer's 3-bit codes back to its bf16 compacted block."""
+    import torch
+    S = len(sides)
+    _need(kq, "kq", at_least=int(kc_rows) * 3 * D // 8)
+    _need(vq, "vq", at_least=int(kc_rows) * 3 * D // 8)
+    for t, nm in ((kc, "kc"), (vc, "vc")):
+        _need(t, nm, at_least=int(kc_rows) * D)
+    _need(k_scale, "k_scale", numel=B * H * S * D)
+    _need(v_scale, "v_scale", numel=B * H * S * D)
+    _need(head_off, "head_off", numel=H)
+    _need(seg_off, "seg_off", numel=H * S)
+    s_arr, s_ptr = _sides_arg(sides)
+    rc = _load().vark_dequantize_layer_int3(
+        _dptr(kq, torch.uint8, "kq"), _dptr(vq, torch.uint8, "vq"), _dptr(k_scale, torch.int16, "k_scale"),
+        _dptr(v_scale, torch.int16, "v_scale"), int(kc_rows), int(B), int(H), len(s_arr), int(D), s_ptr,
+        _dptr(head_off, torch.int32, "head_off"), _dptr(seg_off, torch.int32, "seg_off"),
+        _dptr(kc, torch.bfloat16, "kc"), _dptr(vc, torch.bfloat16, "vc"), _stream(stream))
+    _check(rc, "vark_dequantize_layer_int3")

@@ -425,7 +425,8 @@ __device__ __forceinline__ void absmax8(uint32_t (&acc)[4], const uint4& x) {
 }
 
 // Channel scale: 8-bit codes sc = a / 127 (IEEE); 4-bit codes sc = bf16(a / 7)
-// (IEEE division rounded to bf16, the value the 4-bit scale table stores);
+// and 3-bit codes sc = bf16(a / 3) (IEEE division rounded to bf16, the value the
+// scale table stores);
 // rc = RN(1 / sc) when the product path is usable (2^-100 <= sc <= 2^100),
 // else 0 (always divide).
 struct QScale {
@@ -437,7 +438,7 @@ __device__ __forceinline__ float round_to_bf16(float x) { return __uint_as_float
 template <int BITS>
 __device__ __forceinline__ QScale make_qscale(float a) {
   QScale q;
-  q.sc = BITS == 8 ? a / 127.f : round_to_bf16(a / 7.f);
+  q.sc = BITS == 8 ? a / 127.f : round_to_bf16(a / (BITS == 4 ? 7.f : 3.f));
   q.rc = (q.sc >= 0x1p-100f && q.sc <= 0x1p100f) ? __frcp_rn(q.sc) : 0.f;
   return q;
 }
@@ -465,8 +466,8 @@ __device__ __forceinline__ uint32_t pack4_low_bytes(float y0, float y1, float y2
 
 // y[j] = kRound + rint(x_j / sc_j) for the 8 channels of one 16-byte vector.
 // With 8-bit codes |x / sc| <= 127 (1 + 2^-24); with 4-bit codes sc = bf16(a / 7)
-// >= (a / 7)(1 - 2^-8), so |x / sc| < 7.03: rint never leaves [-127, 127] /
-// [-7, 7] and no clamp is needed.
+// >= (a / 7)(1 - 2^-8), so |x / sc| < 7.03, and with 3-bit codes |x / sc| < 3.02:
+// rint never leaves [-127, 127] / [-7, 7] / [-3, 3] and no clamp is needed.
 __device__ __forceinline__ void code_sums8(const uint4& x, const float (&sc)[8], const float (&rc)[8], bool force,
                                            float (&y)[8]) {
   const float v[8] = {lo_bf16(x.x), hi_bf16(x.x), lo_bf16(x.y), hi_bf16(x.y),
@@ -513,9 +514,28 @@ __device__ __forceinline__ uint32_t codes4x8(const uint4& x, const float (&sc)[8
   return w;
 }
 
+// 3-bit codes: field = code + 4 at bits 3j of a 24-bit group (8 channels, 3
+// bytes, little-endian); the low bits of kRound + code + 4 are the field.
+__device__ __forceinline__ uint32_t codes3x8(const uint4& x, const float (&sc)[8], const float (&rc)[8], bool force) {
+  float y[8];
+  code_sums8(x, sc, rc, force, y);
+  uint32_t w = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) w |= ((__float_as_uint(y[j]) + 4u) & 0x7u) << (3 * j);
+  return w;
+}
+
+__device__ __forceinline__ void store3(uint8_t* p, uint32_t w) {
+  p[0] = uint8_t(w);
+  p[1] = uint8_t(w >> 8);
+  p[2] = uint8_t(w >> 16);
+}
+
 // BITS = 8: kq / vq int8 codes (one byte per element), ka / va fp32 absmax.
 // BITS = 4: kq / vq packed nibbles (one 32-bit word per 8 elements), ka / va
 // bf16 bits (uint16) of the scale bf16(a / 7).
+// BITS = 3: kq / vq 24-bit groups (3 bytes per 8 elements), ka / va bf16 bits
+// of the scale bf16(a / 3).
 template <int BITS>
 __global__ void __cluster_dims__(kQuantCluster, 1, 1) __launch_bounds__(kQuantThreads, 5) quant_kernel(
     const uint4* __restrict__ k, const uint4* __restrict__ v, QuantParams p, const uint8_t* __restrict__ keep,
@@ -646,7 +666,17 @@ __global__ void __cluster_dims__(kQuantCluster, 1, 1) __launch_bounds__(kQuantTh
       // element index of this CTA's first row; 8 elements per 8-byte (int8) or 4-byte (int4) store
       const int64_t e_first = layer_base[q.l] + (row0 + r_lo) * D;
       int32_t r = rg;
-      if (BITS == 8) {
+      if (BITS == 3) {
+        uint8_t* dst = static_cast<uint8_t*>(q.t ? vq : kq) + (e_first / 8) * 3 + cv * 3;
+        for (; r + 3 * nrg < nr; r += 4 * nrg) {
+          uint4 x[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) x[e] = __ldcs(src + (r + e * nrg) * cv_n);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) store3(dst + int64_t(r + e * nrg) * cv_n * 3, codes3x8(x[e], sc, rc, force));
+        }
+        for (; r < nr; r += nrg) store3(dst + int64_t(r) * cv_n * 3, codes3x8(__ldcs(src + r * cv_n), sc, rc, force));
+      } else if (BITS == 8) {
         uint2* dst = reinterpret_cast<uint2*>(static_cast<int8_t*>(q.t ? vq : kq) + e_first) + cv;
         for (; r + 3 * nrg < nr; r += 4 * nrg) {
           uint4 x[4];
@@ -675,7 +705,7 @@ __global__ void __cluster_dims__(kQuantCluster, 1, 1) __launch_bounds__(kQuantTh
         const uint32_t w = fin[c >> 1];
         const float a = (c & 1) ? hi_bf16(w) : lo_bf16(w);
         if (BITS == 8) static_cast<float*>(q.t ? va : ka)[t0 + c] = a;
-        else static_cast<uint16_t*>(q.t ? va : ka)[t0 + c] = uint16_t(__float_as_uint(make_qscale<4>(a).sc) >> 16);
+        else static_cast<uint16_t*>(q.t ? va : ka)[t0 + c] = uint16_t(__float_as_uint(make_qscale<BITS>(a).sc) >> 16);
       }
     }
   }
@@ -699,6 +729,7 @@ struct DequantParams {
 
 // BITS = 8: codes are uint2 per 8 elements, tables fp32 absmax (scale a / 127).
 // BITS = 4: codes are one uint32 word per 8 elements, tables bf16 scale bits.
+// BITS = 3: codes are 3 bytes per 8 elements (a 24-bit group), tables bf16 scale bits.
 template <int BITS>
 __global__ void __launch_bounds__(kDeqThreads, 3) dequant_kernel(const void* __restrict__ kq_,
                                                               const void* __restrict__ vq_,
@@ -708,8 +739,15 @@ __global__ void __launch_bounds__(kDeqThreads, 3) dequant_kernel(const void* __r
                                                               const int32_t* __restrict__ seg_off,
                                                               uint4* __restrict__ kc, uint4* __restrict__ vc) {
   using CodeVec = typename std::conditional<BITS == 8, uint2, uint32_t>::type;
-  const CodeVec* __restrict__ kq = static_cast<const CodeVec*>(kq_);
-  const CodeVec* __restrict__ vq = static_cast<const CodeVec*>(vq_);
+  // code group e (8 elements) of a code buffer
+  auto load_codes = [](const void* base, int64_t e) -> CodeVec {
+    if constexpr (BITS == 3) {
+      const uint8_t* b = static_cast<const uint8_t*>(base) + e * 3;
+      return uint32_t(__ldcs(b)) | (uint32_t(__ldcs(b + 1)) << 8) | (uint32_t(__ldcs(b + 2)) << 16);
+    } else {
+      return __ldcs(static_cast<const CodeVec*>(base) + e);
+    }
+  };
   __shared__ int32_t prefix[kDeqMaxH + 1];
   __shared__ uint32_t masks[kDeqMaxH];
   __shared__ int32_t warp_tot[kDeqThreads / 32];
@@ -765,9 +803,23 @@ __global__ void __launch_bounds__(kDeqThreads, 3) dequant_kernel(const void* __r
     o.w = pack_bf16x2(__fmul_rn(x(w, 12), sc[6]), __fmul_rn(x(w, 28), sc[7]));
     return o;
   };
+  // A 3-bit field f (code + 4) reads 1.5 * 2^23 + f in the same way; the
+  // product code * sc has at most 10 significant bits.
+  auto expand3 = [](uint32_t w, const float (&sc)[8]) {
+    auto x = [](uint32_t u, int shift) {
+      return __fsub_rn(__uint_as_float(0x4B400000u | ((u >> shift) & 0x7u)), 12582916.0f);
+    };
+    uint4 o;
+    o.x = pack_bf16x2(__fmul_rn(x(w, 0), sc[0]), __fmul_rn(x(w, 3), sc[1]));
+    o.y = pack_bf16x2(__fmul_rn(x(w, 6), sc[2]), __fmul_rn(x(w, 9), sc[3]));
+    o.z = pack_bf16x2(__fmul_rn(x(w, 12), sc[4]), __fmul_rn(x(w, 15), sc[5]));
+    o.w = pack_bf16x2(__fmul_rn(x(w, 18), sc[6]), __fmul_rn(x(w, 21), sc[7]));
+    return o;
+  };
   auto expand = [&](CodeVec w, const float (&sc)[8]) {
     if constexpr (BITS == 8) return expand8(w, sc);
-    else return expand4(w, sc);
+    else if constexpr (BITS == 4) return expand4(w, sc);
+    else return expand3(w, sc);
   };
   // units in memory order (batch, head, kept chunk)
   for (int64_t g = blockIdx.x; g < units; g += gridDim.x) {
@@ -819,8 +871,8 @@ __global__ void __launch_bounds__(kDeqThreads, 3) dequant_kernel(const void* __r
       CodeVec ck[4], cw[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        ck[u] = __ldcs(kq + e0 + int64_t(r + u * nrg) * cv_n);
-        cw[u] = __ldcs(vq + e0 + int64_t(r + u * nrg) * cv_n);
+        ck[u] = load_codes(kq_, e0 + int64_t(r + u * nrg) * cv_n);
+        cw[u] = load_codes(vq_, e0 + int64_t(r + u * nrg) * cv_n);
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
@@ -830,8 +882,8 @@ __global__ void __launch_bounds__(kDeqThreads, 3) dequant_kernel(const void* __r
     }
     for (; r < nrows; r += nrg) {
       const int64_t e = e0 + int64_t(r) * cv_n;
-      const CodeVec ck = __ldcs(kq + e);
-      const CodeVec cw = __ldcs(vq + e);
+      const CodeVec ck = load_codes(kq_, e);
+      const CodeVec cw = load_codes(vq_, e);
       kc[e] = expand(ck, sk);
       vc[e] = expand(cw, sv);
     }
@@ -905,7 +957,7 @@ static int dequantize_layer(const void* kq, const void* vq, const void* k_tab, c
   if (rc) return rc;
   if (B < 1 || H < 1 || H > kDeqMaxH || D < 8 || D % 8 != 0 || D > 512 || kc_rows < 0 || kc_rows % B != 0)
     return VARK_E_SHAPE;
-  const uintptr_t code_align = BITS == 8 ? 7 : 3;
+  const uintptr_t code_align = BITS == 8 ? 7 : BITS == 4 ? 3 : 0;
   if (!aligned16(k_tab) || !aligned16(v_tab) || (reinterpret_cast<uintptr_t>(kq) & code_align) ||
       (reinterpret_cast<uintptr_t>(vq) & code_align) || !aligned16(kc) || !aligned16(vc))
     return VARK_E_ALIGN;
@@ -936,6 +988,14 @@ extern "C" int vark_quantize_kv_int4(const uint16_t* k, const uint16_t* v, int64
                         k_scale, v_scale, stream);
 }
 
+extern "C" int vark_quantize_kv_int3(const uint16_t* k, const uint16_t* v, int64_t layer_stride, int L, int B, int H,
+                                     int S, int D, const int32_t* sides, const uint8_t* keep,
+                                     const int32_t* head_off, const int32_t* seg_off, const int64_t* layer_base,
+                                     uint8_t* kq, uint8_t* vq, uint16_t* k_scale, uint16_t* v_scale, void* stream) {
+  return quantize_kv<3>(k, v, layer_stride, L, B, H, S, D, sides, keep, head_off, seg_off, layer_base, kq, vq,
+                        k_scale, v_scale, stream);
+}
+
 extern "C" int vark_dequantize_layer_int8(const int8_t* kq, const int8_t* vq, const float* k_absmax,
                                           const float* v_absmax, int64_t kc_rows, int B, int H, int S, int D,
                                           const int32_t* sides, const int32_t* head_off, const int32_t* seg_off,
@@ -949,5 +1009,13 @@ extern "C" int vark_dequantize_layer_int4(const uint8_t* kq, const uint8_t* vq, 
                                           const int32_t* sides, const int32_t* head_off, const int32_t* seg_off,
                                           uint16_t* kc, uint16_t* vc, void* stream) {
   return dequantize_layer<4>(kq, vq, k_scale, v_scale, kc_rows, B, H, S, D, sides, head_off, seg_off, kc, vc,
+                             stream);
+}
+
+extern "C" int vark_dequantize_layer_int3(const uint8_t* kq, const uint8_t* vq, const uint16_t* k_scale,
+                                          const uint16_t* v_scale, int64_t kc_rows, int B, int H, int S, int D,
+                                          const int32_t* sides, const int32_t* head_off, const int32_t* seg_off,
+                                          uint16_t* kc, uint16_t* vc, void* stream) {
+  return dequantize_layer<3>(kq, vq, k_scale, v_scale, kc_rows, B, H, S, D, sides, head_off, seg_off, kc, vc,
                              stream);
 }

@@ -6,14 +6,18 @@
  *   schedule STATUS k0 k1 ...            (keep[L][H][S])
  *   finalize STATUS x0 x1 ...            (S-CAS of a mass array built from the input)
  *   cache STATUS b0 b1 ...               (bytes[S][L] for B = 2, D = 64)
- *   device STATUS                         (a device call: argument check or no device)
+ *   device STATUS                         (only with the argument "device", given on a
+ *                                         host without a GPU: a device call whose
+ *                                         placeholder pointers would otherwise be used)
  */
 #include <stdio.h>
 #include <stdlib.h>
+#include <string.h>
 
 #include "vark.h"
 
-int main(void) {
+int main(int argc, char** argv) {
+  const int device_call = argc > 1 && strcmp(argv[1], "device") == 0;
   int L, H, S, n_sinks;
   unsigned budget;
   if (scanf("%d %d %d %d %u", &L, &H, &S, &n_sinks, &budget) != 5) return 2;
@@ -56,12 +60,14 @@ int main(void) {
     for (int i = 0; i < S * L; ++i) printf(" %lld", (long long)bytes[i]);
   printf("\n");
 
-  /* a device call with aligned dummy pointers: on a host without a GPU this
-   * reports VARK_E_DEVICE; the strings come from the library */
-  int32_t* dummy = aligned_alloc(64, 4096);
-  rc = vark_build_offsets(keep, L, H, S, sides, 1, 64, dummy, dummy, dummy, (int64_t*)dummy, NULL);
-  printf("device %d %s\n", rc, vark_status_string(rc));
-  free(dummy);
+  /* a device call with aligned placeholder pointers: on a host without a GPU
+   * this reports VARK_E_DEVICE; the strings come from the library */
+  if (device_call) {
+    int32_t* dummy = aligned_alloc(64, 4096);
+    rc = vark_build_offsets(keep, L, H, S, sides, 1, 64, dummy, dummy, dummy, (int64_t*)dummy, NULL);
+    printf("device %d %s\n", rc, vark_status_string(rc));
+    free(dummy);
+  }
   free(scas); free(keep); free(mass); free(fin); free(bytes);
   return 0;
 }

@@ -29,11 +29,18 @@ def exe(tmp_path_factory):
     return out
 
 
+def _no_device():
+    import torch
+    return not torch.cuda.is_available()
+
+
 def _run(exe, scas, sides, n_sinks, budget):
     L, H, S = scas.shape
     text = f"{L} {H} {S} {n_sinks} {budget}\n" + " ".join(map(str, sides)) + "\n" + \
            " ".join(repr(float(x)) for x in scas.ravel()) + "\n"
-    r = subprocess.run([exe], input=text, capture_output=True, text=True, timeout=60)
+    # the device call uses placeholder host pointers: only where no GPU could run it
+    args = [exe, "device"] if _no_device() else [exe]
+    r = subprocess.run(args, input=text, capture_output=True, text=True, timeout=60)
     assert r.returncode == 0, r.stderr
     return {ln.split()[0]: ln.split()[1:] for ln in r.stdout.strip().splitlines()}
 
@@ -57,8 +64,9 @@ def test_c_program_matches_oracle(exe, sides, L, H, budget):
     cache = np.array(list(map(int, out["cache"][1:]))).reshape(S, L)
     assert np.array_equal(cache, oracle.cache_size_after_layer(ref, sides, 2, 64))
     # no GPU here: a device call reports a status from the library's own table
-    status = int(out["device"][0])
-    assert status in (0, -7) and out["device"][1].startswith("VARK")
+    if _no_device():
+        status = int(out["device"][0])
+        assert status == -7 and out["device"][1].startswith("VARK")
 
 
 def test_c_program_reports_infeasible_budget(exe):
