@@ -430,8 +430,9 @@ int vark_dequantize_layer_int4(const uint8_t* kq, const uint8_t* vq, const uint1
 
 /* ---------------------------------------------------------------------------
  * Quantised retained cache (3-bit).  [VAR-Q] summary page, Main Findings: INT3
- * codes on the (block, channel) groups stay within one FID point of BF16; Key
- * Contributions: packing realises the saving (up to 78.5% of the KV cache).
+ * codes on the (block, channel) groups stay within one FID point of BF16 on
+ * the next-scale image models; Key Contributions: packing turns the nominal
+ * bit width into memory savings (the page reports up to 78.5%).
  * Same groups; per channel:
  *   a    = max |x| over the block        s = bf16(a / 3)   (IEEE fp32 division, RNE to bf16)
  *   code = rint(x / s) in [-3, 3]        (IEEE fp32 division, half to even; s = 0 gives 0)
