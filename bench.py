@@ -1024,8 +1024,9 @@ def profile_case(case: str, reps: int):
     counters); 'pruned' = pruned attention of one layer of the 32-layer
     workload (batch 8, 10% budget schedule); 'compact' = compaction of 4
     layers of that workload; 'quant' = int8 quantising compaction of those 4
-    layers, then the dequantisation of each; 'quant4' = 4-bit quantising
-    compaction of those 4 layers, then the dequantisation of each."""
+    layers, then the dequantisation of each; 'quant4' / 'quant3' = 4-bit /
+    3-bit quantising compaction of those 4 layers, then the dequantisation of
+    each."""
     import torch
     import kv_cache_compression_cas_b200 as vark
     dev = torch.device("cuda", 0)
@@ -1058,20 +1059,22 @@ def profile_case(case: str, reps: int):
         kc = torch.empty(max(total, 8), dtype=torch.bfloat16, device=dev)
         vc = torch.empty_like(kc)
         reps_c = reps if case == "compact" else 1
-        if case == "quant4":
-            kq4 = torch.empty(max(total // 2, 16), dtype=torch.uint8, device=dev)
+        if case in ("quant4", "quant3"):
+            num, den = (1, 2) if case == "quant4" else (3, 8)
+            quantize = vark.vark_quantize_kv_int4 if case == "quant4" else vark.vark_quantize_kv_int3
+            dequantize = vark.vark_dequantize_layer_int4 if case == "quant4" else vark.vark_dequantize_layer_int3
+            kq4 = torch.empty(max(num * total // den, 16), dtype=torch.uint8, device=dev)
             vq4 = torch.empty_like(kq4)
             ks4 = torch.empty((L, B, H, S, D), dtype=torch.int16, device=dev)
             vs4 = torch.empty_like(ks4)
             for _ in range(reps):
-                vark.vark_quantize_kv_int4(k, v, B * H * T * D, L, B, H, sides, D, keep_d, ho, so, lb, kq4, vq4, ks4,
-                                           vs4)
+                quantize(k, v, B * H * T * D, L, B, H, sides, D, keep_d, ho, so, lb, kq4, vq4, ks4, vs4)
             base4 = lb.cpu().numpy()
             for _ in range(reps):
                 for l in range(L):
                     rows = int(base4[l + 1] - base4[l]) // D
-                    vark.vark_dequantize_layer_int4(kq4[int(base4[l]) // 2:], vq4[int(base4[l]) // 2:], ks4[l], vs4[l],
-                                                    rows, B, H, sides, D, ho[l], so[l], kc, vc)
+                    b0 = num * int(base4[l]) // den
+                    dequantize(kq4[b0:], vq4[b0:], ks4[l], vs4[l], rows, B, H, sides, D, ho[l], so[l], kc, vc)
             reps_c = 0
         for _ in range(reps_c):
             vark.vark_compact_kv(k, v, B * H * T * D, L, B, H, sides, D, keep_d, ho, so, lb, kc, vc)
@@ -1103,7 +1106,7 @@ def profile_case(case: str, reps: int):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--profile-case", choices=["calib", "calib16", "pruned", "compact", "quant", "quant4"],
+    ap.add_argument("--profile-case", choices=["calib", "calib16", "pruned", "compact", "quant", "quant4", "quant3"],
                     default=None)
     ap.add_argument("--profile-reps", type=int, default=3)
     ap.add_argument("--gpus", type=int, default=1)
