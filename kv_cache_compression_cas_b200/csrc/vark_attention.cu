@@ -67,6 +67,12 @@ constexpr int kPolyPer8 = 0;
 // softmax is bound by MUFU throughput: there 2 of 8 columns on the polynomial
 // measured 12% faster than 0 (4 of 8: 7%).
 constexpr int kPolyPer8NoO = 2;
+// Columns of a full tile exponentiated against the running max before the
+// tile max is known (calibration with O, after the first tile).
+constexpr int kSpecKeys = 64;
+template <int N>
+struct Int { static constexpr int value = N; };
+
 
 struct Params {
   ScaleTable sc;
@@ -552,9 +558,33 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         tc_fence_before();
         mbar_arrive(bar(kBarPFull + x * kPChunks));
       }
-      float m_tile, sh;
+      // Exponent of column c: sv[c] * qk2 + (b2 - m) on a full single-scale
+      // tile (fast), sv[c] * qk2 + colbias[c] - m otherwise.  In calibration
+      // with O, after the first tile, a fast tile's first kSpecKeys columns are
+      // exponentiated against the running max while the tile's row max is
+      // taken alongside, so the max is off the S -> P -> PV -> S chain; a row
+      // whose max grew by more than the threshold (rare after the first
+      // tiles) rescales and recomputes those columns from S_X, which is still
+      // in TMEM.  (Measured +4.5% on calibration, -2% on pruned attention,
+      // which therefore takes the max first.)
+      constexpr int kPoly = WITH_O ? kPolyPer8 : kPolyPer8NoO;
+      auto exp_fast = [&](float* cv, float shift, auto ncols) {
+        constexpr int kN = decltype(ncols)::value;
+#pragma unroll
+        for (int c = 0; c < kN; c += 2) ffma2(cv[c], cv[c + 1], cv[c], cv[c + 1], qk2, qk2, shift, shift);
+#pragma unroll
+        for (int c = 0; c < kN; c += 8) {
+#pragma unroll
+          for (int i = 0; i < kPoly; i += 2) exp2_poly2(cv[c + i], cv[c + i + 1]);
+#pragma unroll
+          for (int i = kPoly; i < 8; ++i) cv[c + i] = ex2_approx(cv[c + i]);
+        }
+      };
+      const bool spec = MASS && WITH_O && fast && j > 0;
+      float b2 = 0.f, m_tile;
       if (fast) {
-        // one source scale, all columns valid: exponent = sv * qk2 + (b2 - m)
+        // one source scale, all columns valid
+        b2 = bias2_sm[seg_scale];
         float m0 = sv[0], m1 = sv[1], m2 = sv[2], m3 = sv[3];
 #pragma unroll
         for (int c = 4; c < kBlockN - 4; c += 8) {
@@ -565,9 +595,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         }
         m0 = fmax3(m0, sv[kBlockN - 4], sv[kBlockN - 3]);
         m1 = fmax3(m1, sv[kBlockN - 2], sv[kBlockN - 1]);
-        const float b2 = bias2_sm[seg_scale];
+        if (spec) exp_fast(sv, b2 - m_used, Int<kSpecKeys>{});   // independent of the max above
         m_tile = fmaf(fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)), qk2, b2);
-        sh = b2;
       } else {
         // boundary / tail tile: per-column bias (or -inf mask) from a table
         // the tile's 128 threads fill, one column each
@@ -591,7 +620,6 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
         m0 = fmax3(m0, sv[kBlockN - 4], sv[kBlockN - 3]);
         m1 = fmax3(m1, sv[kBlockN - 2], sv[kBlockN - 1]);
         m_tile = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
-        sh = 0.f;
       }
       // Running max with a stale-max threshold; O_X is stable here (the
       // commit that completed S_X(j) also covers PV_X(j-1)).
@@ -616,26 +644,32 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
           for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
           tmem_st32(tO + c * 32, v);
         }
+        if (spec) {
+          // chunk 0 went against the old max in the rows that moved: reload
+          // their scores and recompute
+#pragma unroll
+          for (int c = 0; c < kSpecKeys / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tS + c * 32, v);
+            tmem_wait_ld();
+            reg_fence32(v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sv[c * 32 + i] = (f != 1.f) ? __uint_as_float(v[i]) : sv[c * 32 + i];
+          }
+          if (f != 1.f) exp_fast(sv, b2 - m_used, Int<kSpecKeys>{});
+        }
       }
       // p = 2^(exponent - m_used), one chunk of PC::kKeys columns at a time.
       // With O, chunk q's bf16 pairs go to TMEM (over S_X's first columns)
       // while chunk q+1's exponentials run, and the warp signals the chunk
       // to the MMA thread once its store has completed.
-      const float shm = fast ? sh - m_used : -m_used;
+      const float shm = fast ? b2 - m_used : -m_used;
 #pragma unroll
       for (int q = 0; q < PC::kCount; ++q) {
         float* cv = sv + q * PC::kKeys;
         if (fast) {
-#pragma unroll
-          for (int c = 0; c < PC::kKeys; c += 2) ffma2(cv[c], cv[c + 1], cv[c], cv[c + 1], qk2, qk2, shm, shm);
-#pragma unroll
-          for (int c = 0; c < PC::kKeys; c += 8) {
-            constexpr int kPoly = WITH_O ? kPolyPer8 : kPolyPer8NoO;
-#pragma unroll
-            for (int i = 0; i < kPoly; i += 2) exp2_poly2(cv[c + i], cv[c + i + 1]);
-#pragma unroll
-            for (int i = kPoly; i < 8; ++i) cv[c + i] = ex2_approx(cv[c + i]);
-          }
+          if (!(spec && q == 0)) exp_fast(cv, shm, Int<PC::kKeys>{});
+          else exp_fast(cv + kSpecKeys, shm, Int<PC::kKeys - kSpecKeys>{});
         } else {
 #pragma unroll
           for (int c = 0; c < PC::kKeys; c += 2) fadd2(cv[c], cv[c + 1], cv[c], cv[c + 1], shm, shm);
