@@ -58,10 +58,10 @@ constexpr int kPanelBytes = 128 * 128;   // 128 rows x 128 bytes (64 bf16)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 domain
 // Of every 8 columns of a full single-segment tile, this many take 2^x from the
-// FMA-pipe polynomial and the rest from MUFU ex2.  MUFU alone matches the
-// tensor pipe's time per score at D = 128, but measured on B200 the softmax
-// is bound by instruction issue, not MUFU: shares of 2, 4, 6 per 8 ran 5-17%
-// slower than 0, so the polynomial path is off.
+// FMA-pipe polynomial and the rest from MUFU ex2.  With O the tile period is set
+// by the S -> P -> PV -> S chain together with the MMA issuer's bookkeeping,
+// not by MUFU throughput: shares of 2, 4, 6 per 8 ran 5-17% slower than 0,
+// so the polynomial path is off.
 constexpr int kPolyPer8 = 0;
 // Without an output (S-CAS only) there is no P -> PV -> S chain and the
 // softmax is bound by MUFU throughput: there 2 of 8 columns on the polynomial
