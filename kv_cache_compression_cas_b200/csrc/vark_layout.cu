@@ -449,8 +449,10 @@ __device__ __forceinline__ QScale make_qscale(float a) {
 // t = x * rc (rc = RN(1 / sc)) differs from the quotient by at most
 // |t| * 1.5 * 2^-23 (two roundings of relative 2^-24, plus the quotient's own
 // half ulp), so rint(t) = rint(quotient) unless t lies within that distance of
-// a half-integer.  Elements within |t| * 2^-20 of one (ties x = a / 2 are
-// common in bf16 data) take the exact division instead.
+// a half-integer.  Elements whose t lies within 2^-13 of one (a band that
+// contains every |t| * 2^-20 distance, since |t| <= 127 (1 + 2^-23); ties
+// x = a / 2 are common in bf16 data) take the exact division instead.  The
+// product and rounding steps run as packed f32x2 pairs.
 __device__ __forceinline__ float lo_bf16(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float hi_bf16(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
@@ -458,6 +460,10 @@ __device__ __forceinline__ float hi_bf16(uint32_t w) { return __uint_as_float(w 
 // integer (round to nearest, ties to even: the sum's ulp is 1), and the sum's
 // low byte is then that integer's two's-complement byte.
 constexpr float kRound = 12582912.0f;
+// |t| <= 127 (1 + 2^-23) gives |t| * 2^-20 < 2^-13, so every element whose
+// product may round differently from the quotient has |t - rint(t)| above
+// this band.
+constexpr float kTieBand = 0.5f - 0x1p-13f;
 
 __device__ __forceinline__ uint32_t pack4_low_bytes(float y0, float y1, float y2, float y3) {
   return __byte_perm(__byte_perm(__float_as_uint(y0), __float_as_uint(y1), 0x0040),
@@ -472,19 +478,20 @@ __device__ __forceinline__ void code_sums8(const uint4& x, const float (&sc)[8],
                                            float (&y)[8]) {
   const float v[8] = {lo_bf16(x.x), hi_bf16(x.x), lo_bf16(x.y), hi_bf16(x.y),
                       lo_bf16(x.z), hi_bf16(x.z), lo_bf16(x.w), hi_bf16(x.w)};
-  float d[8];         // d > 1/2: t lies within |t| * 2^-20 of a half-integer
+  float t[8], r[8], e[8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const float t = __fmul_rn(v[j], rc[j]);
-    y[j] = __fadd_rn(t, kRound);
-    const float e = __fsub_rn(t, __fsub_rn(y[j], kRound));   // t - rint(t), exact
-    d[j] = fmaf(fabsf(t), 0x1p-20f, fabsf(e));
+  for (int j = 0; j < 8; j += 2) {
+    ffma2(t[j], t[j + 1], v[j], v[j + 1], rc[j], rc[j + 1], 0.f, 0.f);           // t = RN(x * rc)
+    fadd2(y[j], y[j + 1], t[j], t[j + 1], kRound, kRound);                      // kRound + rint(t)
+    fadd2(r[j], r[j + 1], y[j], y[j + 1], -kRound, -kRound);                    // rint(t), exact
+    ffma2(e[j], e[j + 1], r[j], r[j + 1], -1.f, -1.f, t[j], t[j + 1]);           // t - rint(t), exact
   }
-  const float dmax = fmaxf(fmaxf(fmaxf(d[0], d[1]), fmaxf(d[2], d[3])), fmaxf(fmaxf(d[4], d[5]), fmaxf(d[6], d[7])));
-  if (force || dmax > 0.5f) {   // rare: decide the flagged elements by the exact quotient
+  const float emax = fmaxf(fmaxf(fmaxf(fabsf(e[0]), fabsf(e[1])), fmaxf(fabsf(e[2]), fabsf(e[3]))),
+                           fmaxf(fmaxf(fabsf(e[4]), fabsf(e[5])), fmaxf(fabsf(e[6]), fabsf(e[7]))));
+  if (force || emax > kTieBand) {   // rare: decide the flagged elements by the exact quotient
 #pragma unroll
     for (int j = 0; j < 8; ++j)
-      if (force || d[j] > 0.5f) y[j] = __fadd_rn(sc[j] == 0.f ? 0.f : __fdiv_rn(v[j], sc[j]), kRound);
+      if (force || fabsf(e[j]) > kTieBand) y[j] = __fadd_rn(sc[j] == 0.f ? 0.f : __fdiv_rn(v[j], sc[j]), kRound);
   }
 }
 
