@@ -106,7 +106,7 @@ __device__ __forceinline__ void block_exclusive_scan(int32_t* a, int n, int32_t*
 
 constexpr int kChunkRows = 64;
 constexpr int kCompactThreads = 256;
-constexpr int kCompactInflight = 4;
+constexpr int kCompactInflight = 2;   // K + V vectors per thread in flight (2 measured ahead of 4 and 8)
 constexpr int kMaxGroupLH = 4096;   // (layer, head) pairs per launch group
 
 struct CompactParams {
