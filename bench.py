@@ -490,8 +490,9 @@ class CpuSample:
 
 def int8_cache(pipe, max_over_ranks, bf16_attention_ms, hbm_gbs, reps=3):
     """The retained cache stored as int8 codes with per-(block, channel) absmax:
-    quantising compaction of all layers, then per layer dequantisation into a
-    one-layer bf16 buffer followed by that layer's pruned attention."""
+    quantising compaction of all layers, then per layer either dequantisation
+    into a one-layer bf16 buffer followed by that layer's pruned attention, or
+    pruned attention straight over the codes (dequantised in the kernel)."""
     import torch
     vark, w = pipe.vark, pipe.w
     L, B, H, D, S, T = w.layers, w.batch, w.heads, w.head_dim, pipe.S, pipe.T
@@ -506,7 +507,7 @@ def int8_cache(pipe, max_over_ranks, bf16_attention_ms, hbm_gbs, reps=3):
     kcl = torch.empty(max(max_rows * D, 16), dtype=torch.bfloat16, device=dev)
     vcl = torch.empty_like(kcl)
     st = torch.cuda.current_stream()
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
 
     def one():
         ev[0].record(st)
@@ -528,18 +529,27 @@ def int8_cache(pipe, max_over_ranks, bf16_attention_ms, hbm_gbs, reps=3):
             vark.vark_dequantize_layer_int8(kq[b0:], vq[b0:], ka[l], va[l], rows, B, H, pipe.sides, D,
                                             pipe.head_off[l], pipe.seg_off[l], kcl, vcl)
         ev[3].record(st)
+        for l in range(L):     # attention straight over the codes
+            rows = int(base[l + 1] - base[l]) // D
+            b0 = int(base[l])
+            vark.vark_pruned_attention_int8(pipe.q[l], kq[b0:], vq[b0:], ka[l], va[l], rows, pipe.k[l], pipe.v[l],
+                                            pipe.sides, -1, pipe.head_off[l], pipe.seg_off[l], pipe.past_len[l],
+                                            pipe.tau[l], pipe.bias[l], pipe.out[l], pipe.status)
+        ev[4].record(st)
 
     one()
     torch.cuda.synchronize()
-    tq = ta = td = 0.0
+    tq = ta = td = tf = 0.0
     for _ in range(reps):
         one()
         torch.cuda.synchronize()
         tq += ev[0].elapsed_time(ev[1]) / 1e3
         ta += ev[1].elapsed_time(ev[2]) / 1e3
         td += ev[2].elapsed_time(ev[3]) / 1e3
+        tf += ev[3].elapsed_time(ev[4]) / 1e3
     assert int(pipe.status.item()) == 0
     tq, ta, td = max_over_ranks(tq / reps), max_over_ranks(ta / reps), max_over_ranks(td / reps)
+    tf = max_over_ranks(tf / reps)
     bf16_bytes = 2 * 2 * total
     absmax_bytes = 2 * 4 * ka.numel()
     int8_bytes = 2 * total + absmax_bytes
@@ -551,21 +561,23 @@ def int8_cache(pipe, max_over_ranks, bf16_attention_ms, hbm_gbs, reps=3):
             "quantize_gbs": q_bytes / tq / 1e9, "quantize_frac_of_hbm": q_bytes / tq / 1e9 / hbm_gbs,
             "dequantize_ms": td * 1e3, "dequantize_gbs": q_bytes / td / 1e9,
             "dequantize_frac_of_hbm": q_bytes / td / 1e9 / hbm_gbs,
-            "dequant_plus_attention_ms": ta * 1e3,
+            "dequant_plus_attention_ms": ta * 1e3, "fused_attention_ms": tf * 1e3,
             "bf16_cache_attention_ms": bf16_attention_ms}
 
 
 def packed_cache(pipe, max_over_ranks, bf16_attention_ms, hbm_gbs, bits, reps=3):
     """The retained cache stored as packed 4-bit or 3-bit codes with
     per-(block, channel) bf16 scales: quantising compaction of all layers,
-    then per layer dequantisation into a one-layer bf16 buffer followed by
-    that layer's pruned attention."""
+    then per layer either dequantisation into a one-layer bf16 buffer followed
+    by that layer's pruned attention, or pruned attention straight over the
+    codes (dequantised in the kernel)."""
     import torch
     vark, w = pipe.vark, pipe.w
     L, B, H, D, S, T = w.layers, w.batch, w.heads, w.head_dim, pipe.S, pipe.T
     num, den = {4: (1, 2), 3: (3, 8)}[bits]      # code bytes per element
     quantize = {4: vark.vark_quantize_kv_int4, 3: vark.vark_quantize_kv_int3}[bits]
     dequantize = {4: vark.vark_dequantize_layer_int4, 3: vark.vark_dequantize_layer_int3}[bits]
+    fused = {4: vark.vark_pruned_attention_int4, 3: vark.vark_pruned_attention_int3}[bits]
     base = pipe.base_host.numpy()
     total = int(base[-1])
     dev = pipe.dev
@@ -577,7 +589,7 @@ def packed_cache(pipe, max_over_ranks, bf16_attention_ms, hbm_gbs, bits, reps=3)
     kcl = torch.empty(max(max_rows * D, 16), dtype=torch.bfloat16, device=dev)
     vcl = torch.empty_like(kcl)
     st = torch.cuda.current_stream()
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
 
     def one():
         ev[0].record(st)
@@ -599,18 +611,27 @@ def packed_cache(pipe, max_over_ranks, bf16_attention_ms, hbm_gbs, bits, reps=3)
             dequantize(kq[b0:], vq[b0:], ks[l], vs[l], rows, B, H, pipe.sides, D, pipe.head_off[l],
                        pipe.seg_off[l], kcl, vcl)
         ev[3].record(st)
+        for l in range(L):     # attention straight over the codes
+            rows = int(base[l + 1] - base[l]) // D
+            b0 = num * int(base[l]) // den
+            fused(pipe.q[l], kq[b0:], vq[b0:], ks[l], vs[l], rows, pipe.k[l], pipe.v[l], pipe.sides, -1,
+                  pipe.head_off[l], pipe.seg_off[l], pipe.past_len[l], pipe.tau[l], pipe.bias[l], pipe.out[l],
+                  pipe.status)
+        ev[4].record(st)
 
     one()
     torch.cuda.synchronize()
-    tq = ta = td = 0.0
+    tq = ta = td = tf = 0.0
     for _ in range(reps):
         one()
         torch.cuda.synchronize()
         tq += ev[0].elapsed_time(ev[1]) / 1e3
         ta += ev[1].elapsed_time(ev[2]) / 1e3
         td += ev[2].elapsed_time(ev[3]) / 1e3
+        tf += ev[3].elapsed_time(ev[4]) / 1e3
     assert int(pipe.status.item()) == 0
     tq, ta, td = max_over_ranks(tq / reps), max_over_ranks(ta / reps), max_over_ranks(td / reps)
+    tf = max_over_ranks(tf / reps)
     bf16_bytes = 2 * 2 * total
     packed_bytes = 2 * (num * total // den) + 2 * 2 * ks.numel()
     q_bytes = bf16_bytes + packed_bytes   # kept bf16 K, V read once; packed codes and scale tables written
@@ -620,7 +641,8 @@ def packed_cache(pipe, max_over_ranks, bf16_attention_ms, hbm_gbs, bits, reps=3)
             "quantize_frac_of_hbm": q_bytes / tq / 1e9 / hbm_gbs,
             "dequantize_ms": td * 1e3, "dequantize_gbs": q_bytes / td / 1e9,
             "dequantize_frac_of_hbm": q_bytes / td / 1e9 / hbm_gbs,
-            "dequant_plus_attention_ms": ta * 1e3, "bf16_cache_attention_ms": bf16_attention_ms}
+            "dequant_plus_attention_ms": ta * 1e3, "fused_attention_ms": tf * 1e3,
+            "bf16_cache_attention_ms": bf16_attention_ms}
 
 
 def scas_only(pipe, max_over_ranks, with_o_ms, peaks, reps=2):

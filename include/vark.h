@@ -473,6 +473,66 @@ int vark_dequantize_layer_int3(const uint8_t* kq, const uint8_t* vq, const uint1
                                const int32_t* sides, const int32_t* head_off, const int32_t* seg_off,
                                uint16_t* kc, uint16_t* vc, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Pruned attention straight over a quantised retained cache.  [VAR-Q] Why This
+ * Matters: quantisation composes with eviction; here the dequantisation is
+ * part of the attention kernel itself, so no bf16 copy of a layer's cache is
+ * written.  The past K / V tiles are expanded from the codes in shared memory
+ * with exactly the arithmetic of vark_dequantize_layer_int8 / _int4 / _int3,
+ * so the output equals vark_pruned_attention over the dequantised block bit
+ * for bit.
+ * ------------------------------------------------------------------------- */
+
+/*
+ * vark_pruned_attention_int8 -- device.  vark_pruned_attention whose past
+ * comes as this layer's 8-bit codes and absmax tables.
+ *   kq, vq       dev int8, the layer's codes (kq + layer_base[l]), kc_rows
+ *                rows of D bytes; 16-byte aligned.
+ *   k_absmax, v_absmax  dev fp32 [B][H][S][D], the layer's tables (element
+ *                l*B*H*S*D of vark_quantize_kv_int8's); 16-byte aligned.
+ *   other arguments as vark_pruned_attention.
+ * Codes and tables must come from vark_quantize_kv_int8 with the same offset
+ * tables: a past tile whose rows would lie outside [0, kc_rows) is not read
+ * and sets *dev_status to VARK_E_SHAPE.
+ * Errors: as vark_pruned_attention.
+ */
+int vark_pruned_attention_int8(const uint16_t* q, const int8_t* kq, const int8_t* vq,
+                               const float* k_absmax, const float* v_absmax, int64_t kc_rows,
+                               const uint16_t* k_dense, const uint16_t* v_dense,
+                               int B, int H, int S, int D, const int32_t* sides, int query_scale,
+                               const int32_t* head_off, const int32_t* seg_off, const int32_t* past_len,
+                               const float* tau, const float* bias,
+                               uint16_t* out, int32_t* dev_status, void* stream);
+
+/*
+ * vark_pruned_attention_int4 -- device.  As vark_pruned_attention_int8 over
+ * 4-bit codes: kq, vq hold the layer's packed codes (kq + layer_base[l] / 2),
+ * rows of D / 2 bytes; k_scale, v_scale the layer's bf16 scale tables.
+ * Errors: as vark_pruned_attention.
+ */
+int vark_pruned_attention_int4(const uint16_t* q, const uint8_t* kq, const uint8_t* vq,
+                               const uint16_t* k_scale, const uint16_t* v_scale, int64_t kc_rows,
+                               const uint16_t* k_dense, const uint16_t* v_dense,
+                               int B, int H, int S, int D, const int32_t* sides, int query_scale,
+                               const int32_t* head_off, const int32_t* seg_off, const int32_t* past_len,
+                               const float* tau, const float* bias,
+                               uint16_t* out, int32_t* dev_status, void* stream);
+
+/*
+ * vark_pruned_attention_int3 -- device.  As vark_pruned_attention_int4 over
+ * 3-bit codes (kq + 3 layer_base[l] / 8, rows of 3 D / 8 bytes).  A packed
+ * tile is copied whole, so rows must be a multiple of 16 bytes: D = 128 only
+ * (D = 64 returns VARK_E_SHAPE; use vark_dequantize_layer_int3 there).
+ * Errors: as vark_pruned_attention.
+ */
+int vark_pruned_attention_int3(const uint16_t* q, const uint8_t* kq, const uint8_t* vq,
+                               const uint16_t* k_scale, const uint16_t* v_scale, int64_t kc_rows,
+                               const uint16_t* k_dense, const uint16_t* v_dense,
+                               int B, int H, int S, int D, const int32_t* sides, int query_scale,
+                               const int32_t* head_off, const int32_t* seg_off, const int32_t* past_len,
+                               const float* tau, const float* bias,
+                               uint16_t* out, int32_t* dev_status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

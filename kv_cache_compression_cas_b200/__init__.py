@@ -60,6 +60,12 @@ _SIGNATURES = {
     "vark_dequantize_layer_int4": (_I, [_P, _P, _P, _P, _I64, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
     "vark_quantize_kv_int3": (_I, [_P, _P, _I64, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "vark_dequantize_layer_int3": (_I, [_P, _P, _P, _P, _I64, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
+    "vark_pruned_attention_int8": (_I, [_P, _P, _P, _P, _P, _I64, _P, _P, _I, _I, _I, _I, _P, _I, _P, _P, _P, _P,
+                                        _P, _P, _P, _P]),
+    "vark_pruned_attention_int4": (_I, [_P, _P, _P, _P, _P, _I64, _P, _P, _I, _I, _I, _I, _P, _I, _P, _P, _P, _P,
+                                        _P, _P, _P, _P]),
+    "vark_pruned_attention_int3": (_I, [_P, _P, _P, _P, _P, _I64, _P, _P, _I, _I, _I, _I, _P, _I, _P, _P, _P, _P,
+                                        _P, _P, _P, _P]),
 }
 
 
@@ -523,3 +529,62 @@ def vark_dequantize_layer_int3(kq, vq, k_scale, v_scale, kc_rows: int, B: int, H
         _dptr(head_off, torch.int32, "head_off"), _dptr(seg_off, torch.int32, "seg_off"),
         _dptr(kc, torch.bfloat16, "kc"), _dptr(vc, torch.bfloat16, "vc"), _stream(stream))
     _check(rc, "vark_dequantize_layer_int3")
+
+
+def _pruned_packed(bits, q, kq, vq, k_tab, v_tab, kc_rows: int, k_dense, v_dense, sides, query_scale: int,
+                   head_off, seg_off, past_len, tau, bias, out, dev_status, stream):
+    import torch
+    B, H, T, D = _dims(k_dense, 4, "k_dense")
+    S = len(sides)
+    if T != _tokens(sides):
+        raise ValueError(f"k_dense: {T} rows per (batch, head), the scale list has {_tokens(sides)} tokens")
+    if not -1 <= int(query_scale) < S:
+        raise ValueError(f"query_scale {query_scale} out of range")
+    Tq = T if int(query_scale) < 0 else int(sides[query_scale]) ** 2
+    _need(v_dense, "v_dense", shape=(B, H, T, D))
+    _pruned_common_sizes(q, out, None, None, 0, head_off, seg_off, past_len, tau, bias, dev_status,
+                         (B, H, Tq, D), H, S)
+    if int(kc_rows) < 0 or int(kc_rows) % B != 0:
+        raise ValueError(f"kc_rows {kc_rows} must be a non-negative multiple of the batch")
+    code_t, tab_t = (torch.int8, torch.float32) if bits == 8 else (torch.uint8, torch.int16)
+    _need(kq, "kq", at_least=int(kc_rows) * bits * D // 8)
+    _need(vq, "vq", at_least=int(kc_rows) * bits * D // 8)
+    _need(k_tab, "k_tab", numel=B * H * S * D)
+    _need(v_tab, "v_tab", numel=B * H * S * D)
+    s_arr, s_ptr = _sides_arg(sides)
+    fn = getattr(_load(), f"vark_pruned_attention_int{bits}")
+    rc = fn(_dptr(q, torch.bfloat16, "q"), _dptr(kq, code_t, "kq"), _dptr(vq, code_t, "vq"),
+            _dptr(k_tab, tab_t, "k_tab"), _dptr(v_tab, tab_t, "v_tab"), int(kc_rows),
+            _dptr(k_dense, torch.bfloat16, "k_dense"), _dptr(v_dense, torch.bfloat16, "v_dense"),
+            int(B), int(H), len(s_arr), int(D), s_ptr, int(query_scale),
+            _dptr(head_off, torch.int32, "head_off"), _dptr(seg_off, torch.int32, "seg_off"),
+            _dptr(past_len, torch.int32, "past_len"), _dptr(tau, torch.float32, "tau"),
+            _dptr(bias, torch.float32, "bias"), _dptr(out, torch.bfloat16, "out"),
+            _dptr(dev_status, torch.int32, "dev_status"), _stream(stream))
+    _check(rc, f"vark_pruned_attention_int{bits}")
+
+
+def vark_pruned_attention_int8(q, kq, vq, k_absmax, v_absmax, kc_rows: int, k_dense, v_dense, sides,
+                               query_scale: int, head_off, seg_off, past_len, tau, bias, out, dev_status,
+                               stream=None):
+    """Device: pruned attention of one layer straight over its 8-bit codes
+    (kq / vq at the layer's first code, k_absmax / v_absmax the layer's
+    [B][H][S][D] tables); the past is dequantised inside the kernel."""
+    _pruned_packed(8, q, kq, vq, k_absmax, v_absmax, kc_rows, k_dense, v_dense, sides, query_scale, head_off,
+                   seg_off, past_len, tau, bias, out, dev_status, stream)
+
+
+def vark_pruned_attention_int4(q, kq, vq, k_scale, v_scale, kc_rows: int, k_dense, v_dense, sides,
+                               query_scale: int, head_off, seg_off, past_len, tau, bias, out, dev_status,
+                               stream=None):
+    """Device: pruned attention of one layer straight over its packed 4-bit codes."""
+    _pruned_packed(4, q, kq, vq, k_scale, v_scale, kc_rows, k_dense, v_dense, sides, query_scale, head_off,
+                   seg_off, past_len, tau, bias, out, dev_status, stream)
+
+
+def vark_pruned_attention_int3(q, kq, vq, k_scale, v_scale, kc_rows: int, k_dense, v_dense, sides,
+                               query_scale: int, head_off, seg_off, past_len, tau, bias, out, dev_status,
+                               stream=None):
+    """Device: pruned attention of one layer straight over its 3-bit codes (D = 128)."""
+    _pruned_packed(3, q, kq, vq, k_scale, v_scale, kc_rows, k_dense, v_dense, sides, query_scale, head_off,
+                   seg_off, past_len, tau, bias, out, dev_status, stream)

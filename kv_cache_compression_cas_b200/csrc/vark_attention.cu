@@ -93,6 +93,15 @@ struct Params {
   const int32_t* head_off;        // [H]
   const int32_t* seg_off;         // [H][S]
   const int32_t* past_len;        // [H][S]
+  // packed retained past (pruned attention over a quantised cache): this
+  // layer's codes ([kc_rows][D * bits / 8] bytes, K and V) and per-(batch,
+  // head, scale, channel) tables [B][H][S][D] (8-bit: fp32 absmax; 4- and
+  // 3-bit: bf16 scale bits); null otherwise
+  const void* kq;
+  const void* vq;
+  const void* ktab;
+  const void* vtab;
+  int64_t kc_rows;                // rows of the compacted layout (bounds of the code reads)
   // failure-detection test hook (off by default): wait limit, and a key tile
   // the producer withholds so that waits on it run out
   uint64_t wait_limit_ns;
@@ -140,7 +149,13 @@ VARK_DEV void tmem_st_chunk(uint32_t taddr, const uint32_t (&r)[64]) {
   tmem_st32(taddr + 32, reinterpret_cast<const uint32_t(&)[32]>(r[32]));
 }
 
-template <int D>
+// Dynamic shared memory a CTA may opt into on sm_100 (227 KB).
+constexpr int kMaxSmemOptin = 232448;
+
+// Shared-memory layout.  QB = 0: bf16 K/V by TMA.  QB = 8, 4, 3 (pruned
+// attention over a packed past): after the per-CTA tables, the converter's
+// barriers and kCodeSlots staging slots, each holding one K or V tile's codes.
+template <int D, int QB = 0>
 struct Smem {
   static constexpr int kQPanels = D / 64;
   static constexpr int kTile = kQPanels * kPanelBytes;
@@ -155,7 +170,18 @@ struct Smem {
   static constexpr int kSegOff = kBias2 + 32 * 4;       // [32] int32 this head's seg_off (pruned)
   static constexpr int kColBias = kSegOff + 32 * 4;     // [2 tiles][128] fp32 per-column bias / mask
   static constexpr int kMass = kColBias + 2 * 128 * 4;  // [2 tiles][S][128] fp32 (calibration)
-  static int alloc(bool mass, int S) { return kMass + (mass ? 2 * S * kBlockM * 4 : 0) + 1024; }
+  // packed past only (no mass there)
+  static constexpr int kQBar = kMass;                   // [4] converter barriers
+  static constexpr int kCode = kQBar + 128;             // [kCodeSlots] code tiles
+  static constexpr int kCodeRowBytes = D * QB / 8;
+  static constexpr int kSlotBytes = kBlockN * kCodeRowBytes;
+  // two slots where they fit (16 bytes of over-read room for the 3-bit
+  // groups of the last row, 1024 for the base alignment)
+  static constexpr int kCodeSlots = (kCode + 2 * kSlotBytes + 16 + 1024 <= kMaxSmemOptin) ? 2 : 1;
+  static int alloc(bool mass, int S) {
+    if (QB != 0) return kCode + kCodeSlots * kSlotBytes + 16 + 1024;
+    return kMass + (mass ? 2 * S * kBlockM * 4 : 0) + 1024;
+  }
 };
 
 // Tile j of the key list of one work item.
@@ -298,15 +324,208 @@ __device__ __forceinline__ int column_scale(const Params& p, const Item<PRUNED>&
   return it.k;
 }
 
+// ------------------------------------------------------------ packed past
+// Pruned attention over a quantised retained cache (QB = 8, 4 or 3 bits per
+// element in per-(block, channel) groups, as on the VAR-Q summary page, Key
+// Contributions): warps 2 and 3 of the control warpgroup, idle in the bf16
+// kernel, fill the K and V stages of every past tile themselves.  For each K
+// or V tile one thread bulk-copies the tile's packed rows (contiguous in the
+// compacted layout) into a staging slot; the 64 threads then expand every
+// 8-channel group to bf16(code * scale) -- the product in fp32, the same
+// arithmetic as the separate dequantiser, so the tile equals the dequantised
+// cache bit for bit -- and store it in the 128-byte-swizzled layout a TMA
+// load produces.  Rows past the tile's keys are zeros (their columns are
+// masked, and zero V rows keep P * V finite).  Local-scale tiles still come by
+// TMA from the producer.
+//
+// Barrier protocol.  Each stage's "empty" barrier is waited on by the
+// converters for past tiles and by the producer for local tiles, and its
+// "full" barrier gets one arrival per tile from whichever role fills it.  A
+// parity wait is exact only while the waiter is at most one phase behind, so
+// the producer, which skips the past tiles, makes its first stage wait only
+// after the converters have passed all of theirs (kQBarConvDone); from then
+// on the phase it waits for is the current one or the last completed one.
+constexpr int kConvThreads = 64;
+constexpr int kConvBar = 5;          // named barrier of the converter warps
+constexpr int kQBarConvDone = 0;     // the converters are past their last stage wait
+constexpr int kQBarCode = 1;         // [kCodeSlots] a slot's codes have landed
+
+// Eight channels' codes -> four bf16 pairs (channels (0,1) .. (6,7)).  A
+// code's biased value placed in the low mantissa bits of 1.5 * 2^23 reads
+// 1.5 * 2^23 + biased, so one exact subtraction leaves the code; the product
+// with the fp32 scale is rounded to fp32 (exact below 8 bits) and then to bf16.
+template <int QB>
+VARK_DEV uint4 expand_codes(uint32_t w0, uint32_t w1, const float (&sc)[8]) {
+  constexpr float kBias = 12582912.0f + (QB == 8 ? 128.f : QB == 4 ? 8.f : 4.f);
+  uint32_t u[8];
+  if constexpr (QB == 8) {          // bytes 0-3 of w0, then of w1; sign flipped: code + 128
+    const uint32_t a = w0 ^ 0x80808080u, b = w1 ^ 0x80808080u;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      u[i] = __byte_perm(a, 0x4B400000u, 0x7640u | uint32_t(i));
+      u[4 + i] = __byte_perm(b, 0x4B400000u, 0x7640u | uint32_t(i));
+    }
+  } else if constexpr (QB == 4) {   // channel 2i at bit 4i, 2i + 1 at bit 16 + 4i: code + 8
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      u[2 * i] = 0x4B400000u | ((w0 >> (4 * i)) & 0xFu);
+      u[2 * i + 1] = 0x4B400000u | ((w0 >> (16 + 4 * i)) & 0xFu);
+    }
+  } else {                          // channel i at bit 3i of a 24-bit group: code + 4
+#pragma unroll
+    for (int i = 0; i < 8; ++i) u[i] = 0x4B400000u | ((w0 >> (3 * i)) & 0x7u);
+  }
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float c0, c1, v0, v1;
+    fadd2(c0, c1, __uint_as_float(u[2 * i]), __uint_as_float(u[2 * i + 1]), -kBias, -kBias);
+    // + (-0): the plain product, signed zeros included
+    ffma2(v0, v1, c0, c1, sc[2 * i], sc[2 * i + 1], -0.f, -0.f);
+    o[i] = pack_bf16x2(v0, v1);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// The 8 channel scales of one (batch, head, scale) table row from channel
+// 8 * group on: 8-bit tables hold the fp32 absmax a (scale a / 127, IEEE
+// division), 4- and 3-bit tables the bf16 scale bits.
+template <int QB>
+VARK_DEV void load_scales(const void* tab, int64_t idx, float (&sc)[8]) {
+  if constexpr (QB == 8) {
+    const float4* a = reinterpret_cast<const float4*>(static_cast<const float*>(tab) + idx);
+    const float4 x = __ldg(a), y = __ldg(a + 1);
+    sc[0] = x.x / 127.f; sc[1] = x.y / 127.f; sc[2] = x.z / 127.f; sc[3] = x.w / 127.f;
+    sc[4] = y.x / 127.f; sc[5] = y.y / 127.f; sc[6] = y.z / 127.f; sc[7] = y.w / 127.f;
+  } else {
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(tab) + idx));
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      sc[2 * e] = __uint_as_float(ws[e] << 16);
+      sc[2 * e + 1] = __uint_as_float(ws[e] & 0xFFFF0000u);
+    }
+  }
+}
+
+// One K or V past tile from its staged codes into a stage.  Thread ct owns the
+// 8-channel group ct % (D / 8) of every (kConvThreads / (D / 8))-th row; a
+// row's scales are those of the kept scale whose segment holds its key.
+template <int D, int QB>
+VARK_DEV void expand_tile(const Params& p, const Item<true>& it, const KTile& t, const void* tab, uint32_t slot,
+                          uint32_t stage, int ct) {
+  using L = Smem<D, QB>;
+  constexpr int kGroups = D / 8;
+  constexpr int kRowStep = kConvThreads / kGroups;
+  const int cw = ct % kGroups;
+  const uint32_t dst = stage + uint32_t(cw >> 3) * kPanelBytes;   // the group's 64-channel panel
+  const uint32_t chunk = uint32_t(cw & 7);                          // its 16-byte chunk in a row
+  const int S = p.sc.S;
+  const int32_t* segoff = p.seg_off + it.h * S;
+  const int64_t tab0 = (int64_t(it.b) * p.H + it.h) * S * D + cw * 8;
+  int s = -1, seg_hi = -1;   // the kept segment [.., seg_hi) of the current key
+  float sc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+  for (int r = ct / kGroups; r < kBlockN; r += kRowStep) {
+    uint4 o = make_uint4(0u, 0u, 0u, 0u);
+    if (r < t.valid) {
+      const int key = t.key0 + r;
+      if (key >= seg_hi) {
+        do {
+          ++s;
+        } while (s < it.k && (__ldg(segoff + s) < 0 || key >= __ldg(segoff + s) + p.sc.n[s]));
+        seg_hi = __ldg(segoff + s) + p.sc.n[s];
+        load_scales<QB>(tab, tab0 + int64_t(s) * D, sc);
+      }
+      const uint32_t at = slot + uint32_t(r * L::kCodeRowBytes + cw * QB);
+      uint32_t w0, w1 = 0u;
+      if constexpr (QB == 8) {
+        w0 = ld_shared_u32(at);
+        w1 = ld_shared_u32(at + 4);
+      } else if constexpr (QB == 4) {
+        w0 = ld_shared_u32(at);
+      } else {   // a 24-bit group at any byte offset: two aligned words, funnel-shifted
+        w0 = __funnelshift_r(ld_shared_u32(at & ~3u), ld_shared_u32((at & ~3u) + 4u), (at & 3u) * 8u);
+      }
+      o = expand_codes<QB>(w0, w1, sc);
+    }
+    st_shared_v4(dst + uint32_t(r) * 128u + ((chunk ^ uint32_t(r & 7)) << 4), o);
+  }
+}
+
+// The converter role: K then V of past tiles 0 .. n_past - 1, in order.
+template <int D, int QB>
+VARK_DEV void convert_past(const Params& p, const Item<true>& it, uint32_t sK, uint32_t sV, uint32_t sCode,
+                           uint32_t bar0, uint32_t qbar0, volatile int* abort_flag, int ct) {
+  using L = Smem<D, QB>;
+  constexpr int kSlots = L::kCodeSlots;
+  auto bar = [&](int i) { return bar0 + 8u * uint32_t(i); };
+  auto qbar = [&](int i) { return qbar0 + 8u * uint32_t(i); };
+  const int n_conv = p.withhold_tile < 0 ? it.n_past : min(it.n_past, p.withhold_tile);
+  const int U = 2 * n_conv;   // unit u: tile u / 2, K (u even) or V (u odd)
+  // (thread 0) copy of unit u's packed rows into slot u % kSlots
+  auto issue = [&](int u) -> bool {
+    const KTile t = it.tile(p, u >> 1);
+    if (t.row < 0 || int64_t(t.row) + t.valid > p.kc_rows) {   // tables inconsistent with the cache size
+      atomicExch(p.status, VARK_E_SHAPE);
+      *abort_flag = 1;
+      return false;
+    }
+    const int sl = u % kSlots;
+    const uint32_t bytes = uint32_t(t.valid) * uint32_t(L::kCodeRowBytes);
+    const uint8_t* src = static_cast<const uint8_t*>((u & 1) ? p.vq : p.kq) + int64_t(t.row) * L::kCodeRowBytes;
+    mbar_arrive_expect_tx(qbar(kQBarCode + sl), bytes);
+    bulk_load(sCode + uint32_t(sl * L::kSlotBytes), src, bytes, qbar(kQBarCode + sl));
+    return true;
+  };
+  int issued = 0;        // thread 0: units whose copy is issued
+  bool copy_ok = true;
+  if (ct == 0)
+    while (copy_ok && issued < min(U, kSlots)) {
+      copy_ok = issue(issued);
+      if (copy_ok) ++issued;
+    }
+  int u = 0;
+  for (; u < U; ++u) {
+    const int j = u >> 1, which = u & 1, st = j % kStages;
+    // the stage is free once the MMAs of tile j - kStages have read it
+    bool go = j < kStages || mbar_wait(bar((which ? kBarVEmpty : kBarKEmpty) + st), ((j / kStages) - 1) & 1,
+                                       abort_flag, p.status, p.wait_limit_ns);
+    if (!bar_and(kConvBar, kConvThreads, go)) break;
+    if (u == U - 1 && ct == 0) mbar_arrive(qbar(kQBarConvDone));
+    go = mbar_wait(qbar(kQBarCode + u % kSlots), (u / kSlots) & 1, abort_flag, p.status, p.wait_limit_ns);
+    if (!bar_and(kConvBar, kConvThreads, go)) break;
+    expand_tile<D, QB>(p, it, it.tile(p, j), which ? p.vtab : p.ktab, sCode + uint32_t((u % kSlots) * L::kSlotBytes),
+                       (which ? sV : sK) + uint32_t(st * L::kTile), ct);
+    fence_proxy_async_smem();                  // the stage's stores, before the tensor core reads them
+    named_bar_sync(kConvBar, kConvThreads);     // the stage is written and the slot read by all
+    if (ct == 0) {
+      mbar_arrive(bar((which ? kBarVFull : kBarKFull) + st));
+      if (copy_ok && issued < U) {
+        fence_proxy_async_smem();              // the slot's reads, before the copy overwrites it
+        copy_ok = issue(issued);
+        if (copy_ok) ++issued;
+      }
+    }
+  }
+  // Drain (abort path): copies still in flight land before the CTA exits.
+  if (ct == 0) {
+    volatile int no_abort = 0;
+    for (int v = u; v < issued; ++v) mbar_wait(qbar(kQBarCode + v % kSlots), (v / kSlots) & 1, &no_abort, nullptr);
+  }
+}
+
 // WITH_O = false (calibration called without an output): no V tiles and no PV
 // MMAs; the softmax releases S_X as soon as it has read it into registers, so
 // the next S MMA of that tile overlaps the rest of its softmax.
-template <int D, bool PRUNED, bool MASS, bool WITH_O>
+// QB != 0: pruned attention whose past comes as packed codes (converter warps).
+template <int D, bool PRUNED, bool MASS, bool WITH_O, int QB = 0>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kc,
             const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ Params p) {
-  using L = Smem<D>;
+  static_assert(QB == 0 || (PRUNED && WITH_O && !MASS), "packed past: pruned attention only");
+  using L = Smem<D, QB>;
   using PC = PChunks<MASS, WITH_O>;
   constexpr int QP = L::kQPanels;
   constexpr uint32_t kTileBytes = L::kTile;
@@ -342,6 +561,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       mbar_init(bar(kBarODone + x), 1);
     }
     mbar_init(bar(kBarDrain), 1);
+    if constexpr (QB != 0) {
+      mbar_init(sbase + L::kQBar + 8u * kQBarConvDone, 1);
+      for (int sl = 0; sl < L::kCodeSlots; ++sl) mbar_init(sbase + L::kQBar + 8u * (kQBarCode + sl), 1);
+    }
     *abort_flag = 0;
     fence_barrier_init();
     // Start the first loads now, so their latency overlaps TMEM allocation
@@ -361,6 +584,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
     const int first = min(min(n, kStages), p.withhold_tile < 0 ? n : p.withhold_tile);
     for (int j = 0; j < first; ++j) {
       const KTile t = it.tile(p, j);
+      if (QB != 0 && t.src == 1) continue;   // a past tile: the converters fill it
       mbar_arrive_expect_tx(bar(kBarKFull + j), kTileBytes);
       for (int c = 0; c < QP; ++c) {
         const uint32_t dst = sK + j * kTileBytes + c * kPanelBytes;
@@ -393,10 +617,16 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       // barrier initialisation, by this same thread.)
       int issued_k = min(min(n, kStages), p.withhold_tile < 0 ? n : p.withhold_tile);
       int issued_v = WITH_O ? issued_k : 0;
+      bool conv_passed = QB == 0 || it.n_past == 0;   // packed past: the converters' stage waits are behind
       for (int j = issued_k; j < n; ++j) {
         const int st = j % kStages;
         const KTile t = it.tile(p, j);
         if (j == p.withhold_tile) break;   // test hook: this tile never arrives
+        if (QB != 0 && t.src == 1) continue;   // a past tile: the converters fill it
+        if (j >= kStages && !conv_passed) {
+          if (!mbar_wait(sbase + L::kQBar + 8u * kQBarConvDone, 0, abort_flag, p.status, p.wait_limit_ns)) break;
+          conv_passed = true;
+        }
         if (j >= kStages && !mbar_wait(bar(kBarKEmpty + st), ((j / kStages) - 1) & 1, abort_flag, p.status, p.wait_limit_ns)) break;
         mbar_arrive_expect_tx(bar(kBarKFull + st), kTileBytes);
         for (int c = 0; c < QP; ++c) {
@@ -417,11 +647,13 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       }
       // Drain: every load issued here has landed before the CTA exits
       // (immediate on the normal path; bounded on the abort path).
+      // (Past tiles of a packed past are the converters'; they have no copy.)
       volatile int no_abort = 0;
+      const int own0 = QB != 0 ? it.n_past : 0;
       mbar_wait(bar(kBarQ), 0, &no_abort, nullptr);
-      for (int j = max(0, issued_k - kStages); j < issued_k; ++j)
+      for (int j = max(own0, issued_k - kStages); j < issued_k; ++j)
         mbar_wait(bar(kBarKFull + j % kStages), (j / kStages) & 1, &no_abort, nullptr);
-      for (int j = max(0, issued_v - kStages); j < issued_v; ++j)
+      for (int j = max(own0, issued_v - kStages); j < issued_v; ++j)
         mbar_wait(bar(kBarVFull + j % kStages), (j / kStages) & 1, &no_abort, nullptr);
     } else if (warp == 1 && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
@@ -499,6 +731,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CU
       mma_commit(bar(kBarDrain));
       volatile int no_abort = 0;
       mbar_wait(bar(kBarDrain), 0, &no_abort, nullptr);
+    } else if (QB != 0 && (warp == 2 || warp == 3)) {
+      // ---------------------------------------------------------- packed-past converters
+      if constexpr (QB != 0)
+        convert_past<D, QB>(p, it, sK, sV, sbase + L::kCode, bar0, sbase + L::kQBar, abort_flag, threadIdx.x - 64);
     }
   } else {
     setmaxnreg_inc224();
@@ -846,12 +1082,13 @@ static void apply_test_hooks(Params& p) {
   }
 }
 
-template <int D, bool PRUNED, bool MASS, bool WITH_O = true>
+template <int D, bool PRUNED, bool MASS, bool WITH_O = true, int QB = 0>
 static int launch(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& kc,
                   const CUtensorMap& vc, Params& p, cudaStream_t st) {
   apply_test_hooks(p);
-  auto kern = attn_kernel<D, PRUNED, MASS, WITH_O>;
-  const int smem = Smem<D>::alloc(MASS, p.sc.S);
+  auto kern = attn_kernel<D, PRUNED, MASS, WITH_O, QB>;
+  const int smem = Smem<D, QB>::alloc(MASS, p.sc.S);
+  if (smem > kMaxSmemOptin) return VARK_E_SHAPE;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
     cudaGetLastError();
     return VARK_E_CUDA;
@@ -861,9 +1098,6 @@ static int launch(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap&
   kern<<<unsigned(grid), kThreads, smem, st>>>(q, k, v, kc, vc, p);
   return cudaGetLastError() == cudaSuccess ? VARK_OK : VARK_E_CUDA;
 }
-
-// Dynamic shared memory a CTA may opt into on sm_100 (227 KB).
-constexpr int kMaxSmemOptin = 232448;
 
 static bool finite_shape(int B, int H, int T, int D) {
   return B >= 1 && H >= 1 && int64_t(B) * H <= INT32_MAX / 2 && int64_t(B) * H * T * D < (int64_t(1) << 40);
@@ -893,6 +1127,7 @@ extern "C" int vark_scas_accumulate(const uint16_t* q, const uint16_t* k, const 
   lp.tau = tau; lp.bias = bias; lp.mass = mass; lp.out = out; lp.status = dev_status;
   lp.q_rows = lp.sc.T; lp.q_scale_rows = 0; lp.local_scale_only = 0;
   lp.R_l = 0; lp.head_off = nullptr; lp.seg_off = nullptr; lp.past_len = nullptr;
+  lp.kq = lp.vq = lp.ktab = lp.vtab = nullptr; lp.kc_rows = 0;
   if ((rc = build_qtiles(lp, -1))) return rc;
   CUtensorMap tq, tk, tv;
   if ((rc = encode_dense(&tq, q, D, lp.sc.T, int64_t(B) * H))) return rc;
@@ -906,23 +1141,41 @@ extern "C" int vark_scas_accumulate(const uint16_t* q, const uint16_t* k, const 
                   : launch<64, false, true>(tq, tk, tv, tk, tv, lp, st);
 }
 
+// The packed past of a quantised cache (null: bf16 past in kc / vc).
+struct PackedPast {
+  int bits;                 // 8, 4 or 3
+  const void* kq;
+  const void* vq;
+  const void* ktab;
+  const void* vtab;
+};
+
 static int pruned_common(const uint16_t* q, const uint16_t* kc, const uint16_t* vc, int64_t kc_rows,
                          const uint16_t* k_local, const uint16_t* v_local, int B, int H, int S, int D,
                          const int32_t* sides, int query_scale, bool local_scale_only, const int32_t* head_off,
                          const int32_t* seg_off, const int32_t* past_len, const float* tau, const float* bias,
-                         uint16_t* out, int32_t* dev_status, void* stream) {
+                         uint16_t* out, int32_t* dev_status, void* stream, const PackedPast* packed = nullptr) {
   if (!q || !k_local || !v_local || !head_off || !seg_off || !past_len || !tau || !out || !dev_status)
     return VARK_E_ARG;
-  if (kc_rows < 0 || (kc_rows > 0 && (!kc || !vc))) return VARK_E_ARG;
+  if (kc_rows < 0) return VARK_E_ARG;
+  if (packed) {
+    if (kc_rows > 0 && (!packed->kq || !packed->vq || !packed->ktab || !packed->vtab)) return VARK_E_ARG;
+  } else if (kc_rows > 0 && (!kc || !vc)) {
+    return VARK_E_ARG;
+  }
   Params lp;
   int rc = make_scale_table(S, sides, &lp.sc);
   if (rc) return rc;
   if (D != 64 && D != 128) return VARK_E_SHAPE;
+  // a packed K/V tile is copied whole: its rows must be a multiple of 16 bytes
+  if (packed && (D * packed->bits / 8) % 16 != 0) return VARK_E_SHAPE;
   if (query_scale < -1 || query_scale >= S || (local_scale_only && query_scale < 0)) return VARK_E_ARG;
   if (!finite_shape(B, H, lp.sc.T, D)) return VARK_E_SHAPE;
   if (kc_rows % B != 0 || kc_rows > INT32_MAX) return VARK_E_SHAPE;
-  if (!aligned16(q) || !aligned16(k_local) || !aligned16(v_local) || !aligned16(out) ||
-      (kc_rows > 0 && (!aligned16(kc) || !aligned16(vc))))
+  if (!aligned16(q) || !aligned16(k_local) || !aligned16(v_local) || !aligned16(out)) return VARK_E_ALIGN;
+  if (kc_rows > 0 && !packed && (!aligned16(kc) || !aligned16(vc))) return VARK_E_ALIGN;
+  if (kc_rows > 0 && packed &&
+      (!aligned16(packed->kq) || !aligned16(packed->vq) || !aligned16(packed->ktab) || !aligned16(packed->vtab)))
     return VARK_E_ALIGN;
   if ((rc = check_device_sm100())) return rc;
   lp.B = B; lp.H = H;
@@ -933,22 +1186,37 @@ static int pruned_common(const uint16_t* q, const uint16_t* kc, const uint16_t* 
   lp.local_scale_only = local_scale_only ? 1 : 0;
   lp.R_l = kc_rows / B;
   lp.head_off = head_off; lp.seg_off = seg_off; lp.past_len = past_len;
+  lp.kq = packed ? packed->kq : nullptr;
+  lp.vq = packed ? packed->vq : nullptr;
+  lp.ktab = packed ? packed->ktab : nullptr;
+  lp.vtab = packed ? packed->vtab : nullptr;
+  lp.kc_rows = kc_rows;
   if ((rc = build_qtiles(lp, query_scale))) return rc;
   const int64_t local_rows = local_scale_only ? lp.sc.n[query_scale] : lp.sc.T;
   CUtensorMap tq, tk, tv, tkc, tvc;
   if ((rc = encode_dense(&tq, q, D, lp.q_rows, int64_t(B) * H))) return rc;
   if ((rc = encode_dense(&tk, k_local, D, local_rows, int64_t(B) * H))) return rc;
   if ((rc = encode_dense(&tv, v_local, D, local_rows, int64_t(B) * H))) return rc;
-  if (kc_rows > 0) {
+  if (kc_rows > 0 && !packed) {
     if ((rc = encode_rows(&tkc, kc, D, kc_rows))) return rc;
     if ((rc = encode_rows(&tvc, vc, D, kc_rows))) return rc;
   } else {
-    // No head keeps past rows, so these maps are never read; they only need
-    // to be valid 2-D maps.
+    // No head keeps past rows, or the past comes as packed codes: these maps
+    // are never read; they only need to be valid 2-D maps.
     if ((rc = encode_rows(&tkc, k_local, D, 1))) return rc;
     if ((rc = encode_rows(&tvc, v_local, D, 1))) return rc;
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (packed && kc_rows > 0) {
+    switch (packed->bits * 1000 + D) {
+      case 8128: return launch<128, true, false, true, 8>(tq, tk, tv, tkc, tvc, lp, st);
+      case 8064: return launch<64, true, false, true, 8>(tq, tk, tv, tkc, tvc, lp, st);
+      case 4128: return launch<128, true, false, true, 4>(tq, tk, tv, tkc, tvc, lp, st);
+      case 4064: return launch<64, true, false, true, 4>(tq, tk, tv, tkc, tvc, lp, st);
+      case 3128: return launch<128, true, false, true, 3>(tq, tk, tv, tkc, tvc, lp, st);
+      default: return VARK_E_SHAPE;
+    }
+  }
   return D == 128 ? launch<128, true, false>(tq, tk, tv, tkc, tvc, lp, st)
                   : launch<64, true, false>(tq, tk, tv, tkc, tvc, lp, st);
 }
@@ -971,4 +1239,47 @@ extern "C" int vark_pruned_attention_step(const uint16_t* q, const uint16_t* kc,
   if (scale < 0) return VARK_E_ARG;
   return pruned_common(q, kc, vc, kc_rows, k_local, v_local, B, H, S, D, sides, scale, true, head_off, seg_off,
                        past_len, tau, bias, out, dev_status, stream);
+}
+
+// Pruned attention over a quantised retained cache: the past K/V of this
+// layer come as packed codes plus per-(batch, head, scale, channel) tables and
+// are dequantised inside the kernel; no bf16 copy of the cache is written.
+static int pruned_packed(int bits, const uint16_t* q, const void* kq, const void* vq, const void* ktab,
+                         const void* vtab, int64_t kc_rows, const uint16_t* k_dense, const uint16_t* v_dense, int B,
+                         int H, int S, int D, const int32_t* sides, int query_scale, const int32_t* head_off,
+                         const int32_t* seg_off, const int32_t* past_len, const float* tau, const float* bias,
+                         uint16_t* out, int32_t* dev_status, void* stream) {
+  const PackedPast pk = {bits, kq, vq, ktab, vtab};
+  return pruned_common(q, nullptr, nullptr, kc_rows, k_dense, v_dense, B, H, S, D, sides, query_scale, false,
+                       head_off, seg_off, past_len, tau, bias, out, dev_status, stream, &pk);
+}
+
+extern "C" int vark_pruned_attention_int8(const uint16_t* q, const int8_t* kq, const int8_t* vq,
+                                          const float* k_absmax, const float* v_absmax, int64_t kc_rows,
+                                          const uint16_t* k_dense, const uint16_t* v_dense, int B, int H, int S,
+                                          int D, const int32_t* sides, int query_scale, const int32_t* head_off,
+                                          const int32_t* seg_off, const int32_t* past_len, const float* tau,
+                                          const float* bias, uint16_t* out, int32_t* dev_status, void* stream) {
+  return pruned_packed(8, q, kq, vq, k_absmax, v_absmax, kc_rows, k_dense, v_dense, B, H, S, D, sides, query_scale,
+                       head_off, seg_off, past_len, tau, bias, out, dev_status, stream);
+}
+
+extern "C" int vark_pruned_attention_int4(const uint16_t* q, const uint8_t* kq, const uint8_t* vq,
+                                          const uint16_t* k_scale, const uint16_t* v_scale, int64_t kc_rows,
+                                          const uint16_t* k_dense, const uint16_t* v_dense, int B, int H, int S,
+                                          int D, const int32_t* sides, int query_scale, const int32_t* head_off,
+                                          const int32_t* seg_off, const int32_t* past_len, const float* tau,
+                                          const float* bias, uint16_t* out, int32_t* dev_status, void* stream) {
+  return pruned_packed(4, q, kq, vq, k_scale, v_scale, kc_rows, k_dense, v_dense, B, H, S, D, sides, query_scale,
+                       head_off, seg_off, past_len, tau, bias, out, dev_status, stream);
+}
+
+extern "C" int vark_pruned_attention_int3(const uint16_t* q, const uint8_t* kq, const uint8_t* vq,
+                                          const uint16_t* k_scale, const uint16_t* v_scale, int64_t kc_rows,
+                                          const uint16_t* k_dense, const uint16_t* v_dense, int B, int H, int S,
+                                          int D, const int32_t* sides, int query_scale, const int32_t* head_off,
+                                          const int32_t* seg_off, const int32_t* past_len, const float* tau,
+                                          const float* bias, uint16_t* out, int32_t* dev_status, void* stream) {
+  return pruned_packed(3, q, kq, vq, k_scale, v_scale, kc_rows, k_dense, v_dense, B, H, S, D, sides, query_scale,
+                       head_off, seg_off, past_len, tau, bias, out, dev_status, stream);
 }

@@ -295,3 +295,31 @@ def test_int3_calls_reject_bad_arguments_before_the_device():
     # 3-byte groups need no alignment: an odd code pointer passes; kc_rows = 0 returns before any launch
     assert lib.vark_dequantize_layer_int3(ctypes.c_void_p(17), p, p, p, 0, 1, 4, 7, 64, sides, p, p, p, p,
                                           None) in (-7, -5, 0)
+
+
+def test_packed_attention_calls_reject_bad_arguments_before_the_device():
+    lib = vark.library()
+    sides = (ctypes.c_int32 * 7)(*SIDES_TINY)
+    p = ctypes.c_void_p(16)
+    odd = ctypes.c_void_p(24)           # 8-byte but not 16-byte aligned
+
+    def call(bits, q=p, kq=p, tab=p, kc_rows=8, B=1, D=64, qs=-1, dense=p):
+        fn = getattr(lib, f"vark_pruned_attention_int{bits}")
+        return fn(q, kq, p, tab, p, kc_rows, dense, p, B, 4, 7, D, sides, qs, p, p, p, p, None, p, p, None)
+
+    for bits in (8, 4, 3):
+        D = 128 if bits == 3 else 64
+        assert call(bits, q=None, D=D) == -1
+        assert call(bits, kq=None, D=D) == -1          # codes required when a past exists
+        assert call(bits, D=D, qs=7) == -1             # query scale out of range
+        assert call(bits, D=D, kc_rows=9, B=2) == -2   # rows not a multiple of the batch
+        assert call(bits, D=96) == -2                  # head_dim 64 or 128 only
+        assert call(bits, kq=odd, D=D) == -3           # whole tiles are bulk-copied: 16-byte codes
+        assert call(bits, tab=odd, D=D) == -3
+        assert call(bits, dense=odd, D=D) == -3
+    # 3-bit rows of D = 64 are 24 bytes: not a multiple of 16, refused
+    assert call(3, D=64) == -2
+    if _no_device():   # these pass every host check and stop at the device check
+        for bits in (8, 4, 3):
+            assert call(bits, D=128) in (-7, -5)
+            assert call(bits, kq=None, kc_rows=0, D=128) in (-7, -5)   # no past: codes may be absent
