@@ -354,6 +354,29 @@ constexpr int kQBarCode = 1;         // [kCodeSlots] a slot's codes have landed
 // code's biased value placed in the low mantissa bits of 1.5 * 2^23 reads
 // 1.5 * 2^23 + biased, so one exact subtraction leaves the code; the product
 // with the fp32 scale is rounded to fp32 (exact below 8 bits) and then to bf16.
+// 4-bit codes take packed bf16 arithmetic instead: a nibble pair masked into
+// bf16 pairs 128 + n (exponent 2^7, the nibble as the low mantissa bits),
+// minus 136 leaves the codes exactly, and one bf16x2 multiply by the table's
+// scale pair rounds the exact product once -- the same value as the fp32 path.
+VARK_DEV uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+VARK_DEV uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+VARK_DEV uint4 expand_codes4(uint32_t w, const uint32_t (&sp)[4]) {
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t biased = ((w >> (4 * i)) & 0x000F000Fu) | 0x43004300u;   // channel 2i low, 2i + 1 high
+    o[i] = bf16x2_mul(bf16x2_sub(biased, 0x43084308u), sp[i]);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
 template <int QB>
 VARK_DEV uint4 expand_codes(uint32_t w0, uint32_t w1, const float (&sc)[8]) {
   constexpr float kBias = 12582912.0f + (QB == 8 ? 128.f : QB == 4 ? 8.f : 4.f);
@@ -389,7 +412,12 @@ VARK_DEV uint4 expand_codes(uint32_t w0, uint32_t w1, const float (&sc)[8]) {
 
 // The 8 channel scales of one (batch, head, scale) table row from channel
 // 8 * group on: 8-bit tables hold the fp32 absmax a (scale a / 127, IEEE
-// division), 4- and 3-bit tables the bf16 scale bits.
+// division), 4- and 3-bit tables the bf16 scale bits (4-bit: kept as the
+// table's channel pairs, sc unused).
+VARK_DEV void load_scale_pairs(const void* tab, int64_t idx, uint32_t (&sp)[4]) {
+  const uint4 w = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(tab) + idx));
+  sp[0] = w.x; sp[1] = w.y; sp[2] = w.z; sp[3] = w.w;
+}
 template <int QB>
 VARK_DEV void load_scales(const void* tab, int64_t idx, float (&sc)[8]) {
   if constexpr (QB == 8) {
@@ -410,13 +438,16 @@ VARK_DEV void load_scales(const void* tab, int64_t idx, float (&sc)[8]) {
 
 // One K or V past tile from its staged codes into a stage.  Thread ct owns the
 // 8-channel group ct % (D / 8) of every (kConvThreads / (D / 8))-th row; a
-// row's scales are those of the kept scale whose segment holds its key.
+// row's scales are those of the kept scale whose segment holds its key.  Rows
+// go kRowsInFlight at a time: their code loads first, then the expansions.
 template <int D, int QB>
 VARK_DEV void expand_tile(const Params& p, const Item<true>& it, const KTile& t, const void* tab, uint32_t slot,
                           uint32_t stage, int ct) {
   using L = Smem<D, QB>;
   constexpr int kGroups = D / 8;
   constexpr int kRowStep = kConvThreads / kGroups;
+  constexpr int kRowsInFlight = QB == 4 ? 4 : 2;
+  static_assert((kBlockN / kRowStep) % kRowsInFlight == 0, "rows per thread");
   const int cw = ct % kGroups;
   const uint32_t dst = stage + uint32_t(cw >> 3) * kPanelBytes;   // the group's 64-channel panel
   const uint32_t chunk = uint32_t(cw & 7);                          // its 16-byte chunk in a row
@@ -425,31 +456,45 @@ VARK_DEV void expand_tile(const Params& p, const Item<true>& it, const KTile& t,
   const int64_t tab0 = (int64_t(it.b) * p.H + it.h) * S * D + cw * 8;
   int s = -1, seg_hi = -1;   // the kept segment [.., seg_hi) of the current key
   float sc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  uint32_t sp[4] = {0u, 0u, 0u, 0u};
 #pragma unroll 1
-  for (int r = ct / kGroups; r < kBlockN; r += kRowStep) {
-    uint4 o = make_uint4(0u, 0u, 0u, 0u);
-    if (r < t.valid) {
-      const int key = t.key0 + r;
-      if (key >= seg_hi) {
-        do {
-          ++s;
-        } while (s < it.k && (__ldg(segoff + s) < 0 || key >= __ldg(segoff + s) + p.sc.n[s]));
-        seg_hi = __ldg(segoff + s) + p.sc.n[s];
-        load_scales<QB>(tab, tab0 + int64_t(s) * D, sc);
-      }
+  for (int r0 = ct / kGroups; r0 < kBlockN; r0 += kRowsInFlight * kRowStep) {
+    uint32_t w0[kRowsInFlight], w1[kRowsInFlight];
+#pragma unroll
+    for (int i = 0; i < kRowsInFlight; ++i) {
+      const int r = r0 + i * kRowStep;
       const uint32_t at = slot + uint32_t(r * L::kCodeRowBytes + cw * QB);
-      uint32_t w0, w1 = 0u;
-      if constexpr (QB == 8) {
-        w0 = ld_shared_u32(at);
-        w1 = ld_shared_u32(at + 4);
-      } else if constexpr (QB == 4) {
-        w0 = ld_shared_u32(at);
-      } else {   // a 24-bit group at any byte offset: two aligned words, funnel-shifted
-        w0 = __funnelshift_r(ld_shared_u32(at & ~3u), ld_shared_u32((at & ~3u) + 4u), (at & 3u) * 8u);
+      w0[i] = w1[i] = 0u;
+      if (r < t.valid) {
+        if constexpr (QB == 8) {
+          w0[i] = ld_shared_u32(at);
+          w1[i] = ld_shared_u32(at + 4);
+        } else if constexpr (QB == 4) {
+          w0[i] = ld_shared_u32(at);
+        } else {   // a 24-bit group at any byte offset: two aligned words, funnel-shifted
+          w0[i] = __funnelshift_r(ld_shared_u32(at & ~3u), ld_shared_u32((at & ~3u) + 4u), (at & 3u) * 8u);
+        }
       }
-      o = expand_codes<QB>(w0, w1, sc);
     }
-    st_shared_v4(dst + uint32_t(r) * 128u + ((chunk ^ uint32_t(r & 7)) << 4), o);
+#pragma unroll
+    for (int i = 0; i < kRowsInFlight; ++i) {
+      const int r = r0 + i * kRowStep;
+      uint4 o = make_uint4(0u, 0u, 0u, 0u);   // rows past the tile's keys: zeros
+      if (r < t.valid) {
+        const int key = t.key0 + r;
+        if (key >= seg_hi) {
+          do {
+            ++s;
+          } while (s < it.k && (__ldg(segoff + s) < 0 || key >= __ldg(segoff + s) + p.sc.n[s]));
+          seg_hi = __ldg(segoff + s) + p.sc.n[s];
+          if constexpr (QB == 4) load_scale_pairs(tab, tab0 + int64_t(s) * D, sp);
+          else load_scales<QB>(tab, tab0 + int64_t(s) * D, sc);
+        }
+        if constexpr (QB == 4) o = expand_codes4(w0[i], sp);
+        else o = expand_codes<QB>(w0[i], w1[i], sc);
+      }
+      st_shared_v4(dst + uint32_t(r) * 128u + ((chunk ^ uint32_t(r & 7)) << 4), o);
+    }
   }
 }
 

@@ -156,3 +156,49 @@ def test_packed_past_final_scale_query_batch():
     torch.cuda.synchronize()
     assert int(st.item()) == 0, vark.vark_status_string(int(st.item()))
     assert np.array_equal(bits_of(out), bits_of(out_sep))
+
+
+def _scaled_bf16_bits(bits, e):
+    """bf16 bits of x * 2^e (round to nearest even; subnormal results kept)."""
+    f = (f64(bits) * 2.0 ** e).astype(np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    return ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+
+
+@pytest.mark.parametrize("bits,D", [(8, 64), (4, 64), (4, 128), (3, 128)])
+def test_packed_past_subnormal_scales(bits, D):
+    """K and V of magnitude ~2^-128, so every scale and most dequantised values
+    are subnormal: the in-kernel expansion must still equal the dequantiser."""
+    quantize, dequantize, fused, code_t, tab_t, (num, den) = _CALLS[bits]
+    sides, B, H = synth.SIDES_TINY, 2, 2
+    g = oracle.ScaleGeometry(sides)
+    L, T, S = 1, g.T, g.S
+    kb = _scaled_bf16_bits(synth.normal_bf16_bits(synth.derive_key(441, D, 1), (L, B, H, T, D)), -128)
+    vb = _scaled_bf16_bits(synth.normal_bf16_bits(synth.derive_key(441, D, 2), (L, B, H, T, D)), -128)
+    qb = synth.normal_bf16_bits(synth.derive_key(441, D, 3), (B, H, T, D))
+    keep = np.ones((L, H, S), dtype=np.uint8)
+    tab = Tables(keep, sides, B, D)
+    kd, vd, qd = dev_bf16(kb), dev_bf16(vb), dev_bf16(qb)
+    kq = torch.empty(max(num * tab.total // den, 16), dtype=code_t, device="cuda")
+    vq = torch.empty_like(kq)
+    kt = torch.empty((L, B, H, S, D), dtype=tab_t, device="cuda")
+    vt = torch.empty_like(kt)
+    quantize(kd, vd, B * H * T * D, L, B, H, sides, D, tab.keep, tab.head_off, tab.seg_off, tab.layer_base,
+             kq, vq, kt, vt)
+    rows = tab.kc_rows(0)
+    tau = torch.from_numpy(synth.gen_tau(442, H)).cuda()
+    st = status_word()
+    kc = torch.zeros(rows * D, dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    dequantize(kq, vq, kt[0], vt[0], rows, B, H, sides, D, tab.head_off[0], tab.seg_off[0], kc, vc)
+    out_sep = torch.empty_like(qd)
+    vark.vark_pruned_attention(qd, kc, vc, rows, kd[0], vd[0], sides, -1, tab.head_off[0], tab.seg_off[0],
+                               tab.past_len[0], tau, None, out_sep, st)
+    out = torch.full_like(qd, float("nan"))
+    fused(qd, kq, vq, kt[0], vt[0], rows, kd[0], vd[0], sides, -1, tab.head_off[0], tab.seg_off[0],
+          tab.past_len[0], tau, None, out, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0, vark.vark_status_string(int(st.item()))
+    vals = f64(bits_of(vc)[:rows * D])
+    assert np.any((vals != 0) & (np.abs(vals) < 2.0 ** -126))   # the case is really subnormal
+    assert np.array_equal(bits_of(out), bits_of(out_sep))
