@@ -15,6 +15,9 @@
  *   [AMS-KV] "AMS-KV: Adaptive KV Caching in Multi-Scale Visual
  *            Autoregressive Transformers" listing: Abstract (attending to the
  *            local scale matters most; condensed early scales).
+ *   [VAR-Q]  VAR-Q summary page: Key Contributions ((block, channel)
+ *            quantisation groups, bit packing), Main Findings (INT4 / INT3
+ *            quality), Why This Matters (composes with eviction).
  *
  * Conventions shared by every call
  *   - bf16 tensors are passed as `const uint16_t*` holding raw bf16 bits.
