@@ -1004,15 +1004,19 @@ def summarize_kernels(kernels, quant, quant4, quant3, others, scas_o, peaks):
         out["scas_only_qk_tflops"] = r(scas_o["qk_tflops"])
     if quant:
         out["int8"] = {"cache_ratio": r(quant["cache_ratio"]), "quantize_frac_of_hbm": r(quant["quantize_frac_of_hbm"]),
-                       "dequantize_frac_of_hbm": r(quant["dequantize_frac_of_hbm"])}
+                       "dequantize_frac_of_hbm": r(quant["dequantize_frac_of_hbm"]),
+                       "dequant_plus_attention_vs_bf16": r(quant["dequant_plus_attention_ms"] / quant["bf16_cache_attention_ms"]),
+                       "fused_attention_vs_bf16": r(quant["fused_attention_ms"] / quant["bf16_cache_attention_ms"])}
     if quant4:
         out["int4"] = {"cache_ratio": r(quant4["cache_ratio"]), "quantize_frac_of_hbm": r(quant4["quantize_frac_of_hbm"]),
                        "dequantize_frac_of_hbm": r(quant4["dequantize_frac_of_hbm"]),
-                       "dequant_plus_attention_vs_bf16": r(quant4["dequant_plus_attention_ms"] / quant4["bf16_cache_attention_ms"])}
+                       "dequant_plus_attention_vs_bf16": r(quant4["dequant_plus_attention_ms"] / quant4["bf16_cache_attention_ms"]),
+                       "fused_attention_vs_bf16": r(quant4["fused_attention_ms"] / quant4["bf16_cache_attention_ms"])}
     if quant3:
         out["int3"] = {"cache_ratio": r(quant3["cache_ratio"]), "quantize_frac_of_hbm": r(quant3["quantize_frac_of_hbm"]),
                        "dequantize_frac_of_hbm": r(quant3["dequantize_frac_of_hbm"]),
-                       "dequant_plus_attention_vs_bf16": r(quant3["dequant_plus_attention_ms"] / quant3["bf16_cache_attention_ms"])}
+                       "dequant_plus_attention_vs_bf16": r(quant3["dequant_plus_attention_ms"] / quant3["bf16_cache_attention_ms"]),
+                       "fused_attention_vs_bf16": r(quant3["fused_attention_ms"] / quant3["bf16_cache_attention_ms"])}
     if others:
         l8 = others["large_8l"]
         out["large_8l"] = {"calibration_tflops": r(l8["calibration_tflops"]), "pruned_tflops": r(l8["pruned_attention_tflops"]),
