@@ -323,3 +323,33 @@ def test_packed_attention_calls_reject_bad_arguments_before_the_device():
         for bits in (8, 4, 3):
             assert call(bits, D=128) in (-7, -5)
             assert call(bits, kq=None, kc_rows=0, D=128) in (-7, -5)   # no past: codes may be absent
+
+
+def test_binding_refuses_mismatched_packed_attention_sizes():
+    """The attention-over-codes wrappers check codes, tables and the usual
+    query / table sizes before any pointer is taken (CPU tensors)."""
+    import torch
+    sides = SIDES_TINY
+    S, T, D, B, H, rows = 7, 155, 64, 2, 4, 20
+    bf, i32 = torch.bfloat16, torch.int32
+    q = torch.zeros((B, H, T, D), dtype=bf)
+    base = dict(q=q, kc_rows=rows, k_dense=q, v_dense=q, sides=sides, query_scale=-1,
+                head_off=torch.zeros(H, dtype=i32), seg_off=torch.zeros(H, S, dtype=i32),
+                past_len=torch.zeros(H, S, dtype=i32), tau=torch.zeros(H), bias=torch.zeros(H, S), out=q,
+                dev_status=torch.zeros(1, dtype=i32))
+    cases = {
+        8: (vark.vark_pruned_attention_int8, "k_absmax", "v_absmax", torch.int8, torch.float32, rows * D),
+        4: (vark.vark_pruned_attention_int4, "k_scale", "v_scale", torch.uint8, torch.int16, rows * D // 2),
+        3: (vark.vark_pruned_attention_int3, "k_scale", "v_scale", torch.uint8, torch.int16, rows * 3 * D // 8),
+    }
+    for bits, (fn, kt, vt, code_t, tab_t, nbytes) in cases.items():
+        good = {**base, "kq": torch.zeros(nbytes, dtype=code_t), "vq": torch.zeros(nbytes, dtype=code_t),
+                kt: torch.zeros(B * H * S * D, dtype=tab_t), vt: torch.zeros(B * H * S * D, dtype=tab_t)}
+        for key, bad in (("kq", torch.zeros(nbytes - 1, dtype=code_t)), ("vq", torch.zeros(nbytes - 1, dtype=code_t)),
+                         (kt, torch.zeros(B * H * S * D - 1, dtype=tab_t)), ("kc_rows", rows + 1),
+                         ("q", torch.zeros((B, H, T - 1, D), dtype=bf)), ("past_len", torch.zeros(H, dtype=i32)),
+                         ("query_scale", S)):
+            with pytest.raises(ValueError):
+                fn(**{**good, key: bad})
+        with pytest.raises(TypeError):      # sizes right: the device check refuses a CPU tensor
+            fn(**good)
