@@ -102,3 +102,60 @@ def test_code_byte_to_float_by_mantissa_placement():
             bits = _byte_perm(w ^ 0x80808080, 0x4B400000, 0x7640 | pos)
             v = F32(np.array([bits], dtype=np.uint32).view(np.float32)[0] - F32(12583040.0))
             assert v == F32(k)
+
+
+# ---- the same rule with the 4- and 3-bit scales
+# The kernels use one code path for every width: t = RN(x * RN(1 / sc)),
+# y = RN(t + 1.5 * 2^23), the exact quotient where |t - rint(t)| > 1/2 - 2^-13,
+# and the field taken from the low bits of y's pattern plus the bias (8 or 4).
+# With sc = bf16(a / 7) or bf16(a / 3) the band still holds every element whose
+# product may round differently (|t| < 7.03 resp. 3.02).
+
+def _bf16_round(x):
+    """fp32 -> fp32 value of its bf16 rounding (nearest, ties to even)."""
+    b = np.asarray(x, dtype=np.float32).reshape(-1).view(np.uint32).astype(np.uint64)
+    r = ((b + 0x7FFF + ((b >> 16) & 1)) >> 16) << 16
+    return r.astype(np.uint32).view(np.float32).reshape(np.shape(x))
+
+
+def _kernel_rule_packed(x, a, bits):
+    qmax, bias, mask = (7, 8, 0xF) if bits == 4 else (3, 4, 0x7)
+    sc = F32(_bf16_round(F32(a / F32(qmax))))
+    usable = F32(2.0 ** -100) <= sc <= F32(2.0 ** 100)
+    rc = F32(F32(1.0) / sc) if usable else F32(0.0)
+    with np.errstate(over="ignore", invalid="ignore"):
+        t = (x * rc).astype(np.float32)
+        y = (t + K_ROUND).astype(np.float32)
+        r = (y - K_ROUND).astype(np.float32)
+        e = (t - r).astype(np.float32)
+    near = (np.abs(e) > F32(0.5 - 2.0 ** -13)) | (not usable and sc != 0)
+    if near.any():
+        with np.errstate(divide="ignore", invalid="ignore"):
+            q = (x[near] / sc).astype(np.float32) if sc != 0 else np.zeros(int(near.sum()), np.float32)
+        y[near] = (q + K_ROUND).astype(np.float32)
+    field = (y.view(np.uint32) + np.uint32(bias)) & np.uint32(mask)
+    return field.astype(np.int32) - bias, int(near.sum())
+
+
+def _check_absmax_packed(a_bits, bits):
+    from oracle.quant import quantize_block_int3, quantize_block_int4
+    pos = _bf16_bits_upto(a_bits)
+    col = np.concatenate([pos, pos | np.uint16(0x8000)])
+    ref_codes, _ = (quantize_block_int4 if bits == 4 else quantize_block_int3)(col.reshape(-1, 1))
+    a = _f32(np.array([a_bits], dtype=np.uint16))[0]
+    got, n_near = _kernel_rule_packed(_f32(col), a, bits)
+    assert np.array_equal(got, ref_codes[:, 0].astype(np.int32)), (bits, hex(int(a_bits)))
+    return n_near, col.size
+
+
+def test_product_rule_equals_ieee_quotient_packed_widths():
+    for bits in (4, 3):
+        near = total = 0
+        for e_bits in (0x3F80, 0x2000, 0x5F00):
+            for m in range(128):
+                n, t = _check_absmax_packed(e_bits | m, bits)
+                near += n
+                total += t
+        assert 0 < near < total // 20, bits    # ties x = s * (k + 1/2) exist and take the exact path
+        for a_bits in (0x0000, 0x0001, 0x0080, 0x7F7F):
+            _check_absmax_packed(a_bits, bits)
