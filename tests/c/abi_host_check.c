@@ -6,6 +6,7 @@
  *   schedule STATUS k0 k1 ...            (keep[L][H][S])
  *   finalize STATUS x0 x1 ...            (S-CAS of a mass array built from the input)
  *   cache STATUS b0 b1 ...               (bytes[S][L] for B = 2, D = 64)
+ *   args A B C                           (argument errors of three device calls)
  *   device STATUS                         (only with the argument "device", given on a
  *                                         host without a GPU: a device call whose
  *                                         placeholder pointers would otherwise be used)
@@ -59,6 +60,25 @@ int main(int argc, char** argv) {
   if (rc == VARK_OK)
     for (int i = 0; i < S * L; ++i) printf(" %lld", (long long)bytes[i]);
   printf("\n");
+
+  /* argument errors of the attention-over-codes calls come back before any
+   * device work, on any host: a missing query, 3-bit rows of 24 bytes
+   * (D = 64), and 8-bit codes off the 16-byte boundary */
+  {
+    static _Alignas(16) unsigned char buf[256];
+    const uint16_t* p = (const uint16_t*)buf;
+    uint16_t* o = (uint16_t*)buf;
+    int32_t* st = (int32_t*)buf;
+    const int32_t* t = (const int32_t*)buf;
+    const float* f = (const float*)buf;
+    int a = vark_pruned_attention_int4(NULL, buf, buf, p, p, 8, p, p, 1, 1, S, 128, sides, -1, t, t, t, f, NULL, o,
+                                       st, NULL);
+    int b = vark_pruned_attention_int3(p, buf, buf, p, p, 8, p, p, 1, 1, S, 64, sides, -1, t, t, t, f, NULL, o, st,
+                                       NULL);
+    int c = vark_pruned_attention_int8(p, (const int8_t*)(buf + 8), (const int8_t*)buf, f, f, 8, p, p, 1, 1, S, 64,
+                                       sides, -1, t, t, t, f, NULL, o, st, NULL);
+    printf("args %d %d %d\n", a, b, c);
+  }
 
   /* a device call with aligned placeholder pointers: on a host without a GPU
    * this reports VARK_E_DEVICE; the strings come from the library */

@@ -63,6 +63,8 @@ def test_c_program_matches_oracle(exe, sides, L, H, budget):
     assert out["cache"][0] == "0"
     cache = np.array(list(map(int, out["cache"][1:]))).reshape(S, L)
     assert np.array_equal(cache, oracle.cache_size_after_layer(ref, sides, 2, 64))
+    # argument errors of device calls come back before any device work, from C too
+    assert out["args"] == ["-1", "-2", "-3"]
     # no GPU here: a device call reports a status from the library's own table
     if _no_device():
         status = int(out["device"][0])
